@@ -1,0 +1,189 @@
+/*
+ * dmuon.h -- C ABI of the B200 (sm_100a) Muon / DMuon optimizer step.
+ *
+ * One call updates a set of 2-D weight matrices in place.  For every matrix
+ * (rows x cols, row-major, contiguous):
+ *
+ *   B' = mu*B + G                      momentum buffer, in place
+ *   U  = G + mu*B'                     Nesterov look-ahead (nesterov = 1)
+ *   X  = U, or U^T when rows > cols    iterate on the wide orientation
+ *   X0 = X / (||X||_F + eps)
+ *   K times:  A = X X^T,  X <- a X + (b A + c A^2) X        (quintic NS)
+ *   O  = X_K (transposed back)
+ *   W' = (1 - lr*wd) W - lr * 0.2*sqrt(max(rows, cols)) * O
+ *
+ * Sources (page title, section):
+ *   "DeepSpeed 現已支援 Muon Optimizer" (setupai.cc), 技術深入: Muon
+ *     orthogonalises the momentum-based update of 2-D weights by
+ *     Newton-Schulz iterations, with decoupled weight decay and a
+ *     per-parameter scale chosen by RMS matching so AdamW's lr/wd carry over.
+ *   DMuon release article (wjxwpt.net), section 2 "shape-adaptive execution
+ *     stack": the NS iteration may run in the m x m Gram space, small
+ *     matrices are grouped to fill the GPU, and the math form and kernel are
+ *     chosen per shape; section 3: each shape group's full computation is
+ *     measured once and the measured costs drive the work order.
+ *   DMuon announcement (m.zaocj.com), "自變量三招": on a new shape the
+ *     candidate kernels are timed, the best is kept and reused for that shape.
+ * The pages fix neither the coefficients nor eps; the defaults are
+ * (a, b, c) = (3.4445, -4.7750, 2.0315), eps = 1e-7, K = 5.
+ *
+ * Conventions for every entry point:
+ *   - Device pointers are CUDA device memory of the current device; the
+ *     pointer ARRAYS (params, grads, ...) and `shapes` are HOST memory, read
+ *     during the call only.  The caller owns every buffer it passes.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *     asynchronous on it.  The first call that meets a new shape group
+ *     autotunes it and synchronises `stream` (see dmuon_step).
+ *   - Return 0 on success, a negative DMUON_ERR_* code on failure;
+ *     dmuon_last_error() gives a message (thread-local).  Any error detected
+ *     before the first launch leaves every caller buffer untouched.
+ *   - Aliasing between params, grads and momenta of any matrices is
+ *     undefined.  NaN/Inf in a gradient propagates into that matrix only.
+ *   - Calls are serialised per device inside the library; GPU work of two
+ *     calls is ordered through an internal event, so calls on different
+ *     streams are safe.
+ */
+#ifndef DMUON_H
+#define DMUON_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DMUON_VERSION 1
+
+/* Status codes. */
+#define DMUON_OK 0
+#define DMUON_ERR_INVALID (-1)        /* null pointer, bad shape/count/steps, non-finite hyperparameter */
+#define DMUON_ERR_DTYPE (-2)          /* unsupported dtype combination */
+#define DMUON_ERR_CUDA (-3)           /* a CUDA runtime/driver call failed */
+#define DMUON_ERR_OOM (-4)            /* workspace allocation failed or caller workspace too small */
+#define DMUON_ERR_DEVICE_TIMEOUT (-5) /* a bounded device-side wait ran out (pipeline stalled) */
+
+/* Element types. */
+typedef enum dmuon_dtype { DMUON_BF16 = 0, DMUON_F32 = 1 } dmuon_dtype;
+
+/* Newton-Schulz form.  AUTO lets the per-shape autotuner choose. */
+typedef enum dmuon_variant {
+  DMUON_VARIANT_AUTO = 0,
+  DMUON_VARIANT_DIRECT = 1,  /* iterate on X (m x n): 5 x (m^2 n + m^3 + m^2 n) GEMMs */
+  DMUON_VARIANT_GRAM = 2,    /* iterate on Q (m x m), one m x m x n product at the end */
+  DMUON_VARIANT_BATCHED = 3  /* one CTA per small matrix, everything resident on chip */
+} dmuon_variant;
+
+/* Options of dmuon_step_ex.  Zero-initialise, then call dmuon_options_init. */
+typedef struct dmuon_options {
+  int param_dtype;   /* dmuon_dtype of W   (default DMUON_BF16) */
+  int grad_dtype;    /* dmuon_dtype of G   (default DMUON_BF16) */
+  int mom_dtype;     /* dmuon_dtype of B   (default DMUON_F32; only F32 supported) */
+  float eps;         /* added to ||X||_F    (default 1e-7) */
+  int nesterov;      /* 1: U = G + mu*B'; 0: U = B'  (default 1) */
+  int variant;       /* dmuon_variant      (default AUTO) */
+  float ns_a, ns_b, ns_c; /* quintic coefficients (default 3.4445, -4.7750, 2.0315) */
+} dmuon_options;
+
+/* Fill `opts` with the defaults listed above. */
+void dmuon_options_init(dmuon_options* opts);
+
+/*
+ * dmuon_step -- one Muon step over `count` matrices, bf16 params and grads,
+ * fp32 momenta.
+ *   params[i]  device, rows_i x cols_i row-major, bf16; updated in place.
+ *   grads[i]   device, same shape, bf16; read only.
+ *   momenta[i] device, same shape, fp32; updated in place (B').
+ *   shapes     host, 2*count int64: shapes[2i] = rows_i, shapes[2i+1] = cols_i.
+ *   count      >= 0; 0 returns DMUON_OK without work.
+ *   lr, wd, mu finite floats; ns_steps in [0, 16].
+ * Matrices are grouped by (rows, cols); each group is planned once per
+ * process (variant and tiles chosen by timing candidates on that group's
+ * data; this first call synchronises `stream` and writes nothing to the
+ * caller's buffers while timing) and groups run in descending measured cost.
+ */
+int dmuon_step(void* const* params, const void* const* grads, void* const* momenta,
+               const int64_t* shapes, int count, float lr, float wd, float mu,
+               int ns_steps, void* stream);
+
+/* dmuon_step with explicit dtypes and options.  opts == NULL means defaults.
+ * Supported: param/grad both BF16 (tensor-core path, bf16 operands, fp32
+ * accumulate) or both F32 (fp32 SIMT path); momenta F32. */
+int dmuon_step_ex(void* const* params, const void* const* grads, void* const* momenta,
+                  const int64_t* shapes, int count, float lr, float wd, float mu,
+                  int ns_steps, const dmuon_options* opts, void* stream);
+
+/*
+ * dmuon_compute_update -- everything but the parameter write: updates the
+ * momenta like dmuon_step and writes the orthogonalised update O (before the
+ * 0.2*sqrt(max) scale) to out[i], device fp32, rows_i x cols_i row-major.
+ * For parity tests and for callers that apply O themselves.
+ */
+int dmuon_compute_update(const void* const* grads, void* const* momenta,
+                         const int64_t* shapes, int count, float mu, int ns_steps,
+                         const dmuon_options* opts, float* const* out, void* stream);
+
+/*
+ * dmuon_gemm_bf16 -- the tensor-core GEMM core on its own (tests, tuning):
+ *   D[l] = alpha * A[l] * op(B[l]) + beta * C[l]            l = 0..batch-1
+ * A: device bf16, M x K row-major (K contiguous), leading dim lda, batch
+ *    stride sa (elements).  B: device bf16; b_kmajor = 1: stored N x K
+ *    (op(B) = B^T), b_kmajor = 0: stored K x N (op(B) = B).  C, D: device
+ *    bf16 M x N (C may be NULL => beta ignored).  All leading dims and batch
+ *    strides must be multiples of 8 elements and pointers 16-byte aligned.
+ *    bn selects the tile width (128 or 256; 0 = default).
+ */
+int dmuon_gemm_bf16(const void* A, int64_t lda, int64_t sa, const void* B, int64_t ldb,
+                    int64_t sb, int b_kmajor, const void* C, int64_t ldc, int64_t sc,
+                    void* D, int64_t ldd, int64_t sd, int M, int N, int K, int batch,
+                    float alpha, float beta, int bn, void* stream);
+
+/* Autotune cache: save / load (text, one line per shape key, keyed also by
+ * GPU name, SM count and library version) and clear. */
+int dmuon_cache_save(const char* path);
+int dmuon_cache_load(const char* path);
+void dmuon_cache_clear(void);
+
+/* Number of cached shape keys, and the plan of key `i` as text
+ * ("rows cols dtype variant bn chunk cost_ms") into buf (NUL-terminated). */
+int dmuon_cache_size(void);
+int dmuon_cache_entry(int i, char* buf, size_t len);
+
+/*
+ * dmuon_set_workspace -- use a caller-owned device buffer of `bytes` bytes
+ * (256-byte aligned) as scratch instead of the library's own allocation.
+ * NULL / 0 returns to library-managed scratch.  A call whose plan needs more
+ * than `bytes` fails with DMUON_ERR_OOM before any launch.
+ */
+int dmuon_set_workspace(void* dev_ptr, size_t bytes);
+
+/* Scratch bytes the library would need for this set of shapes (planning
+ * only, no allocation, no launch). */
+int dmuon_workspace_size(const int64_t* shapes, int count, int param_dtype, size_t* bytes);
+
+/*
+ * Kernel timing for benchmarks.  While enabled, the library brackets every
+ * launch with CUDA events on the stream it launches on.  dmuon_timing_get
+ * synchronises those events and returns, for kernel class `kind`
+ * (0 = tensor-core GEMM, 1 = momentum/normalise, 2 = SIMT GEMM, 3 = other),
+ * the number of launches, their summed device time in ms, the algorithmic
+ * FLOPs (GEMM: 2*M*N*K*batch) and algorithmic bytes (elementwise kernels).
+ */
+void dmuon_timing_enable(int enable);
+void dmuon_timing_reset(void);
+int dmuon_timing_get(int kind, int64_t* launches, double* ms, double* flops, double* bytes);
+
+/* Number of kernels the library launched since load (all kinds). */
+int64_t dmuon_launch_count(void);
+
+/* Thread-local message of the last error ("" if none). */
+const char* dmuon_last_error(void);
+
+/* DMUON_VERSION of the loaded library. */
+int dmuon_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DMUON_H */

@@ -1,0 +1,256 @@
+"""ctypes binding of ``libdmuon.so`` (the C ABI in ``include/dmuon.h``).
+
+Argument marshalling only: torch tensors are turned into device pointers,
+shapes into an int64 array and the current torch stream into a cudaStream_t.
+Every step of the computation runs in the library's CUDA kernels.  If the
+library is missing this module raises on import: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from pathlib import Path
+
+LIB_PATH = Path(os.environ.get("DMUON_LIB", Path(__file__).resolve().parent / "libdmuon.so"))
+
+DMUON_OK = 0
+DMUON_ERR_INVALID = -1
+DMUON_ERR_DTYPE = -2
+DMUON_ERR_CUDA = -3
+DMUON_ERR_OOM = -4
+DMUON_ERR_DEVICE_TIMEOUT = -5
+
+DMUON_BF16 = 0
+DMUON_F32 = 1
+
+VARIANTS = {"auto": 0, "direct": 1, "gram": 2, "batched": 3}
+KIND_TC_GEMM, KIND_EW, KIND_SIMT_GEMM, KIND_OTHER = 0, 1, 2, 3
+
+# every entry point include/dmuon.h declares
+EXPORTS = (
+    "dmuon_options_init", "dmuon_step", "dmuon_step_ex", "dmuon_compute_update",
+    "dmuon_gemm_bf16", "dmuon_cache_save", "dmuon_cache_load", "dmuon_cache_clear",
+    "dmuon_cache_size", "dmuon_cache_entry", "dmuon_set_workspace", "dmuon_workspace_size",
+    "dmuon_timing_enable", "dmuon_timing_reset", "dmuon_timing_get", "dmuon_launch_count",
+    "dmuon_last_error", "dmuon_version",
+)
+
+
+class DmuonError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"dmuon error {code}: {msg}")
+        self.code = code
+
+
+class Options(ctypes.Structure):
+    _fields_ = [
+        ("param_dtype", ctypes.c_int), ("grad_dtype", ctypes.c_int), ("mom_dtype", ctypes.c_int),
+        ("eps", ctypes.c_float), ("nesterov", ctypes.c_int), ("variant", ctypes.c_int),
+        ("ns_a", ctypes.c_float), ("ns_b", ctypes.c_float), ("ns_c", ctypes.c_float),
+    ]
+
+
+def _load() -> ctypes.CDLL:
+    if not LIB_PATH.exists():
+        raise ImportError(f"{LIB_PATH} not found: build it with `python -m newton_schulz_normalise_b200.build`")
+    lib = ctypes.CDLL(str(LIB_PATH))
+    P, I, F, I64, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int64, ctypes.c_size_t
+    PP = ctypes.POINTER(ctypes.c_void_p)
+    PI64 = ctypes.POINTER(ctypes.c_int64)
+    sig = {
+        "dmuon_options_init": (None, [ctypes.POINTER(Options)]),
+        "dmuon_step": (I, [PP, PP, PP, PI64, I, F, F, F, I, P]),
+        "dmuon_step_ex": (I, [PP, PP, PP, PI64, I, F, F, F, I, ctypes.POINTER(Options), P]),
+        "dmuon_compute_update": (I, [PP, PP, PI64, I, F, I, ctypes.POINTER(Options), PP, P]),
+        "dmuon_gemm_bf16": (I, [P, I64, I64, P, I64, I64, I, P, I64, I64, P, I64, I64, I, I, I, I, F, F, I, P]),
+        "dmuon_cache_save": (I, [ctypes.c_char_p]),
+        "dmuon_cache_load": (I, [ctypes.c_char_p]),
+        "dmuon_cache_clear": (None, []),
+        "dmuon_cache_size": (I, []),
+        "dmuon_cache_entry": (I, [I, ctypes.c_char_p, S]),
+        "dmuon_set_workspace": (I, [P, S]),
+        "dmuon_workspace_size": (I, [PI64, I, I, ctypes.POINTER(S)]),
+        "dmuon_timing_enable": (None, [I]),
+        "dmuon_timing_reset": (None, []),
+        "dmuon_timing_get": (I, [I, PI64, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double),
+                                 ctypes.POINTER(ctypes.c_double)]),
+        "dmuon_launch_count": (I64, []),
+        "dmuon_last_error": (ctypes.c_char_p, []),
+        "dmuon_version": (I, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def last_error() -> str:
+    return lib.dmuon_last_error().decode()
+
+
+def _check(rc: int):
+    if rc != DMUON_OK:
+        raise DmuonError(rc, last_error())
+    return rc
+
+
+def _ptrs(tensors):
+    arr = (ctypes.c_void_p * max(len(tensors), 1))()
+    for i, t in enumerate(tensors):
+        arr[i] = t.data_ptr() if t is not None else None
+    return arr
+
+
+def _shapes(tensors):
+    arr = (ctypes.c_int64 * max(2 * len(tensors), 1))()
+    for i, t in enumerate(tensors):
+        if t.dim() != 2 or not t.is_contiguous():
+            raise ValueError(f"matrix {i}: expected a contiguous 2-D tensor, got {tuple(t.shape)}")
+        arr[2 * i], arr[2 * i + 1] = t.shape
+    return arr
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return DMUON_BF16
+    if t.dtype == torch.float32:
+        return DMUON_F32
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def options(param_dtype=DMUON_BF16, grad_dtype=DMUON_BF16, eps=None, nesterov=None, variant="auto",
+            coeffs=None) -> Options:
+    o = Options()
+    lib.dmuon_options_init(ctypes.byref(o))
+    o.param_dtype, o.grad_dtype = param_dtype, grad_dtype
+    if eps is not None:
+        o.eps = eps
+    if nesterov is not None:
+        o.nesterov = int(nesterov)
+    o.variant = VARIANTS[variant] if isinstance(variant, str) else int(variant)
+    if coeffs is not None:
+        o.ns_a, o.ns_b, o.ns_c = coeffs
+    return o
+
+
+def dmuon_step(params, grads, momenta, lr, wd, mu, ns_steps=5, stream=None):
+    """In-place Muon step over lists of bf16 params/grads and fp32 momenta."""
+    n = len(params)
+    assert len(grads) == n and len(momenta) == n
+    return _check(lib.dmuon_step(_ptrs(params), _ptrs(grads), _ptrs(momenta), _shapes(params), n,
+                                 lr, wd, mu, ns_steps, _stream(stream)))
+
+
+def dmuon_step_ex(params, grads, momenta, lr, wd, mu, ns_steps=5, opts: Options | None = None, stream=None,
+                  **kw):
+    """In-place Muon step with explicit options (dtypes taken from the tensors)."""
+    n = len(params)
+    assert len(grads) == n and len(momenta) == n
+    if opts is None:
+        opts = options(_dtype_code(params[0]) if n else DMUON_BF16,
+                       _dtype_code(grads[0]) if n else DMUON_BF16, **kw)
+    return _check(lib.dmuon_step_ex(_ptrs(params), _ptrs(grads), _ptrs(momenta), _shapes(grads), n,
+                                    lr, wd, mu, ns_steps, ctypes.byref(opts), _stream(stream)))
+
+
+def dmuon_compute_update(grads, momenta, out, mu, ns_steps=5, opts: Options | None = None, stream=None, **kw):
+    """Momentum update + orthogonalised update O (fp32) into ``out`` tensors."""
+    n = len(grads)
+    assert len(momenta) == n and len(out) == n
+    if opts is None:
+        dt = _dtype_code(grads[0]) if n else DMUON_BF16
+        opts = options(dt, dt, **kw)
+    return _check(lib.dmuon_compute_update(_ptrs(grads), _ptrs(momenta), _shapes(grads), n, mu, ns_steps,
+                                           ctypes.byref(opts), _ptrs(out), _stream(stream)))
+
+
+def dmuon_gemm_bf16(A, B, D, alpha=1.0, beta=0.0, C=None, b_kmajor=True, bn=0, stream=None):
+    """D = alpha * A @ op(B) + beta * C on 2-D or 3-D (batched) bf16 tensors."""
+    def geom(t):
+        if t.dim() == 2:
+            return 1, t.shape[0], t.shape[1], t.stride(0), t.shape[0] * t.stride(0)
+        return t.shape[0], t.shape[1], t.shape[2], t.stride(1), t.stride(0)
+    batch, M, K, lda, sa = geom(A)
+    _, b0, b1, ldb, sb = geom(B)
+    N = b0 if b_kmajor else b1
+    _, _, _, ldd, sd = geom(D)
+    ldc = sc = 0
+    if C is not None:
+        _, _, _, ldc, sc = geom(C)
+    return _check(lib.dmuon_gemm_bf16(A.data_ptr(), lda, sa, B.data_ptr(), ldb, sb, int(b_kmajor),
+                                      C.data_ptr() if C is not None else None, ldc, sc,
+                                      D.data_ptr(), ldd, sd, M, N, K, batch, alpha, beta, bn, _stream(stream)))
+
+
+def dmuon_cache_save(path: str):
+    return _check(lib.dmuon_cache_save(str(path).encode()))
+
+
+def dmuon_cache_load(path: str):
+    return _check(lib.dmuon_cache_load(str(path).encode()))
+
+
+def dmuon_cache_clear():
+    lib.dmuon_cache_clear()
+
+
+def dmuon_cache_entries():
+    out = []
+    buf = ctypes.create_string_buffer(256)
+    for i in range(lib.dmuon_cache_size()):
+        _check(lib.dmuon_cache_entry(i, buf, 256))
+        out.append(buf.value.decode())
+    return out
+
+
+def dmuon_set_workspace(tensor_or_none):
+    if tensor_or_none is None:
+        return _check(lib.dmuon_set_workspace(None, 0))
+    t = tensor_or_none
+    return _check(lib.dmuon_set_workspace(t.data_ptr(), t.numel() * t.element_size()))
+
+
+def dmuon_workspace_size(shapes, param_dtype=DMUON_BF16) -> int:
+    arr = (ctypes.c_int64 * max(2 * len(shapes), 1))()
+    for i, (r, c) in enumerate(shapes):
+        arr[2 * i], arr[2 * i + 1] = r, c
+    out = ctypes.c_size_t(0)
+    _check(lib.dmuon_workspace_size(arr, len(shapes), param_dtype, ctypes.byref(out)))
+    return out.value
+
+
+def dmuon_timing_enable(on: bool = True):
+    lib.dmuon_timing_enable(int(on))
+
+
+def dmuon_timing_reset():
+    lib.dmuon_timing_reset()
+
+
+def dmuon_timing_get(kind: int):
+    n = ctypes.c_int64(0)
+    ms, fl, by = ctypes.c_double(0), ctypes.c_double(0), ctypes.c_double(0)
+    _check(lib.dmuon_timing_get(kind, ctypes.byref(n), ctypes.byref(ms), ctypes.byref(fl), ctypes.byref(by)))
+    return {"launches": n.value, "ms": ms.value, "flops": fl.value, "bytes": by.value}
+
+
+def dmuon_launch_count() -> int:
+    return lib.dmuon_launch_count()
+
+
+def dmuon_version() -> int:
+    return lib.dmuon_version()

@@ -1,0 +1,1057 @@
+// dmuon_api.cu -- host side of the Muon step: validation, shape groups,
+// per-shape autotune cache, scratch layout and the Newton-Schulz drivers
+// behind the C ABI of include/dmuon.h.
+//
+// Shape-adaptive execution (DMuon release article, wjxwpt.net, section 2
+// "shape-adaptive execution stack"; DMuon announcement, m.zaocj.com,
+// "自變量三招"): matrices are grouped by shape; the first time a shape key is
+// met, every candidate (direct or Gram-space Newton-Schulz, tile width) runs
+// on that group's own data into scratch, is timed with CUDA events, and must
+// agree with the direct form within a gate before it can win; the winner and
+// its measured cost are cached and reused for that key.  Section 3 of the
+// same article measures each shape group's full computation once and uses
+// the costs to order work; on one GPU the groups are issued in descending
+// measured cost.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <map>
+#include <memory>
+#include <mutex>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "../../include/dmuon.h"
+#include "internal.h"
+
+namespace dmuon {
+namespace {
+
+// ------------------------------------------------------------------ errors
+thread_local std::string t_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_err = buf;
+  if (getenv("DMUON_TRACE")) fprintf(stderr, "[dmuon] error %d: %s\n", code, buf);
+  return code;
+}
+
+#define CUDA_TRY(expr)                                                                          \
+  do {                                                                                          \
+    cudaError_t e__ = (expr);                                                                   \
+    if (e__ != cudaSuccess) return fail(DMUON_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(e__)); \
+  } while (0)
+
+bool trace_on() {
+  static int v = getenv("DMUON_TRACE") ? 1 : 0;
+  return v != 0;
+}
+
+// ------------------------------------------------------------------ timing
+struct TimedLaunch {
+  int kind;
+  cudaEvent_t a, b;
+  double flops, bytes;
+};
+std::mutex g_tmu;
+std::atomic<int> g_timing{0};
+std::vector<TimedLaunch> g_timed;
+std::vector<cudaEvent_t> g_event_pool;
+std::atomic<long long> g_launches{0};
+
+cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Runs `launch` (which enqueues one kernel on `s`), bracketed by events when
+// timing is enabled.
+template <class F>
+cudaError_t launch_k(int kind, double flops, double bytes, cudaStream_t s, F&& launch) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (!g_timing.load(std::memory_order_relaxed)) return launch();
+  std::lock_guard<std::mutex> lk(g_tmu);
+  TimedLaunch t{kind, take_event(), take_event(), flops, bytes};
+  cudaEventRecord(t.a, s);
+  cudaError_t e = launch();
+  cudaEventRecord(t.b, s);
+  g_timed.push_back(t);
+  return e;
+}
+
+// ------------------------------------------------------------------ device context
+struct DeviceCtx {
+  int device = -1;
+  int num_sms = 148;
+  std::string name;
+  std::mutex mu;
+  void* ws = nullptr;  // scratch
+  size_t ws_bytes = 0;
+  bool ws_external = false;
+  void* ext_ptr = nullptr;
+  size_t ext_bytes = 0;
+  // pinned staging for pointer tables (two slots, reused after their copy)
+  void* pin[2] = {nullptr, nullptr};
+  size_t pin_cap[2] = {0, 0};
+  cudaEvent_t pin_ev[2] = {nullptr, nullptr};
+  bool pin_used[2] = {false, false};
+  int pin_next = 0;
+  cudaEvent_t last_done = nullptr;
+  bool has_last = false;
+  int* err_host = nullptr;  // mapped pinned word the kernels write on timeout
+  int* err_dev = nullptr;
+  cudaEvent_t tune_a = nullptr, tune_b = nullptr;
+};
+
+std::mutex g_ctx_mu;
+std::map<int, std::unique_ptr<DeviceCtx>> g_ctx;
+void* g_ext_ptr = nullptr;  // dmuon_set_workspace (applies to the current device)
+size_t g_ext_bytes = 0;
+
+int get_ctx(DeviceCtx** out) {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(g_ctx_mu);
+  auto it = g_ctx.find(dev);
+  if (it == g_ctx.end()) {
+    auto c = std::make_unique<DeviceCtx>();
+    c->device = dev;
+    cudaDeviceProp prop;
+    CUDA_TRY(cudaGetDeviceProperties(&prop, dev));
+    c->num_sms = prop.multiProcessorCount;
+    c->name = prop.name;
+    if (prop.major != 10) return fail(DMUON_ERR_CUDA, "device %d (%s, sm_%d%d) is not an sm_100 GPU", dev, prop.name, prop.major, prop.minor);
+    CUDA_TRY(cudaEventCreateWithFlags(&c->last_done, cudaEventDisableTiming));
+    CUDA_TRY(cudaEventCreateWithFlags(&c->pin_ev[0], cudaEventDisableTiming));
+    CUDA_TRY(cudaEventCreateWithFlags(&c->pin_ev[1], cudaEventDisableTiming));
+    CUDA_TRY(cudaEventCreate(&c->tune_a));
+    CUDA_TRY(cudaEventCreate(&c->tune_b));
+    CUDA_TRY(cudaHostAlloc(reinterpret_cast<void**>(&c->err_host), sizeof(int), cudaHostAllocMapped));
+    *c->err_host = 0;
+    CUDA_TRY(cudaHostGetDevicePointer(reinterpret_cast<void**>(&c->err_dev), c->err_host, 0));
+    it = g_ctx.emplace(dev, std::move(c)).first;
+  }
+  *out = it->second.get();
+  return DMUON_OK;
+}
+
+bool fault_alloc() {
+  const char* f = getenv("DMUON_FAULT");
+  return f && strstr(f, "alloc");
+}
+
+int ensure_ws(DeviceCtx& c, size_t bytes, cudaStream_t s) {
+  if (g_ext_ptr) {
+    if (bytes > g_ext_bytes)
+      return fail(DMUON_ERR_OOM, "caller workspace too small: need %zu bytes, have %zu", bytes, g_ext_bytes);
+    c.ws = g_ext_ptr;
+    c.ws_bytes = g_ext_bytes;
+    c.ws_external = true;
+    return DMUON_OK;
+  }
+  if (c.ws_external) {  // returned to library-managed scratch
+    c.ws = nullptr;
+    c.ws_bytes = 0;
+    c.ws_external = false;
+  }
+  if (bytes <= c.ws_bytes) return DMUON_OK;
+  if (fault_alloc()) return fail(DMUON_ERR_OOM, "injected allocation failure (DMUON_FAULT=alloc)");
+  CUDA_TRY(cudaStreamSynchronize(s));
+  if (c.ws) {
+    CUDA_TRY(cudaDeviceSynchronize());
+    CUDA_TRY(cudaFree(c.ws));
+    c.ws = nullptr;
+    c.ws_bytes = 0;
+  }
+  size_t want = bytes + (bytes >> 4);  // 6% headroom for the next plan
+  cudaError_t e = cudaMalloc(&c.ws, want);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    c.ws = nullptr;
+    return fail(DMUON_ERR_OOM, "cudaMalloc(%zu) for scratch failed: %s", want, cudaGetErrorString(e));
+  }
+  c.ws_bytes = want;
+  return DMUON_OK;
+}
+
+// ------------------------------------------------------------------ plans
+struct Plan {
+  int variant = DMUON_VARIANT_DIRECT;
+  int bn = 256;
+  double cost_ms = 0.0;  // measured for one chunk of `chunk` matrices
+};
+
+struct Key {
+  long long rows, cols;
+  int f32, steps, cnt;
+  bool operator<(const Key& o) const {
+    return std::tie(rows, cols, f32, steps, cnt) < std::tie(o.rows, o.cols, o.f32, o.steps, o.cnt);
+  }
+};
+
+std::mutex g_cache_mu;
+std::map<Key, Plan> g_cache;
+
+// Geometry of one matrix in its wide orientation.
+struct Geo {
+  int rows, cols;  // stored
+  int m, n;        // iterate: m = min, n = max
+  bool transposed;
+  long long ldx, ldm;  // row strides (elements) of X (m x n) and of m x m buffers
+  int esz;             // bytes per element of the iterate
+  long long x_elems() const { return static_cast<long long>(m) * ldx; }
+  long long q_elems() const { return static_cast<long long>(m) * ldm; }
+};
+
+Geo make_geo(long long rows, long long cols, bool f32) {
+  Geo g;
+  g.rows = static_cast<int>(rows);
+  g.cols = static_cast<int>(cols);
+  g.transposed = rows > cols;
+  g.m = static_cast<int>(std::min(rows, cols));
+  g.n = static_cast<int>(std::max(rows, cols));
+  g.ldx = (g.n + 7) / 8 * 8;
+  g.ldm = (g.m + 7) / 8 * 8;
+  g.esz = f32 ? 4 : 2;
+  return g;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Scratch layout of one chunk of `cnt` matrices.
+struct Layout {
+  size_t X0, Xp, Xq, A, Bm, P, Q0, Q1, T, partials, s, s2, total;
+};
+
+Layout make_layout(const Geo& g, int cnt, int nblk) {
+  Layout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t xb = static_cast<size_t>(cnt) * g.x_elems() * g.esz;
+  const size_t qb = static_cast<size_t>(cnt) * g.q_elems() * g.esz;
+  L.X0 = take(xb);
+  L.Xp = take(xb);
+  L.Xq = take(xb);
+  L.A = take(qb);
+  L.Bm = take(qb);
+  L.P = take(qb);
+  L.Q0 = take(qb);
+  L.Q1 = take(qb);
+  L.T = L.Bm;  // T and the direct form's polynomial buffer are never live together
+  L.partials = take(static_cast<size_t>(cnt) * nblk * sizeof(float));
+  L.s = take(static_cast<size_t>(cnt) * sizeof(float));
+  L.s2 = take(static_cast<size_t>(cnt) * sizeof(float));
+  L.total = off;
+  return L;
+}
+
+size_t per_matrix_bytes(const Geo& g) { return 3 * g.x_elems() * g.esz + 5 * g.q_elems() * g.esz + 64; }
+
+size_t budget_bytes() {
+  const char* b = getenv("DMUON_WS_BUDGET_MB");
+  size_t mb = b ? static_cast<size_t>(atoll(b)) : 8192;
+  return mb << 20;
+}
+
+int chunk_size(const Geo& g, int count) {
+  size_t per = per_matrix_bytes(g);
+  size_t c = budget_bytes() / std::max<size_t>(per, 1);
+  if (c < 1) c = 1;
+  if (c > 65535) c = 65535;
+  return static_cast<int>(std::min<size_t>(c, count));
+}
+
+// ------------------------------------------------------------------ NS driver
+struct Hyper {
+  float mu, lr, wd, eps, a, b, c;
+  int steps, nesterov;
+};
+
+struct Chunk {
+  const Geo* g;
+  int cnt;
+  uint8_t* base;  // scratch of this chunk
+  Layout L;
+  void* const* Gt;  // device pointer tables for this chunk
+  void* const* Bt;
+  void* const* Wt;
+  float* const* Ot;
+  int nblk;
+  int aligned;
+};
+
+template <class T>
+T* at(const Chunk& ch, size_t off) {
+  return reinterpret_cast<T*>(ch.base + off);
+}
+
+// One GEMM of the NS recursion.  A: M x K rows (ld lda), B: K-major (N x K)
+// or MN-major (K x N).  Dispatches to tensor cores (bf16) or SIMT (fp32).
+int gemm(DeviceCtx& c, const Geo& g, int cnt, bool f32, int bn, const void* A, long long lda, long long sa,
+         const void* B, long long ldb, long long sb, bool b_kmajor, int M, int N, int K, const Epilogue& e,
+         cudaStream_t s) {
+  const double flops = 2.0 * M * N * static_cast<double>(K) * cnt;
+  cudaError_t err;
+  if (!f32) {
+    TcGemm t{A, lda, sa, B, ldb, sb, b_kmajor, M, N, K, cnt, bn, e};
+    err = launch_k(KIND_TC_GEMM, flops, 0.0, s, [&] { return launch_tc_gemm(t, s, c.err_dev, c.num_sms); });
+  } else {
+    SimtGemm t{static_cast<const float*>(A), lda, sa, static_cast<const float*>(B), ldb, sb, b_kmajor, M, N, K, cnt, e};
+    err = launch_k(KIND_SIMT_GEMM, flops, 0.0, s, [&] { return launch_simt_gemm(t, s); });
+  }
+  if (err != cudaSuccess) return fail(DMUON_ERR_CUDA, "gemm %dx%dx%d (batch %d) launch failed: %s", M, N, K, cnt, cudaGetErrorString(err));
+  (void)g;
+  return DMUON_OK;
+}
+
+Epilogue store_epi(void* D, long long ldd, long long sd, bool f32, float alpha, const float* alpha_vec) {
+  Epilogue e{};
+  e.mode = EPI_STORE;
+  e.alpha = alpha;
+  e.alpha_vec = alpha_vec;
+  e.D = D;
+  e.ldd = ldd;
+  e.sd = sd;
+  e.d_f32 = f32;
+  e.c_f32 = f32;
+  return e;
+}
+
+// Runs K1 (momentum + norm partials) and the finalize for a chunk.
+int run_momentum(DeviceCtx& c, const Chunk& ch, bool f32, bool g_f32, const Hyper& h, cudaStream_t s) {
+  const Geo& g = *ch.g;
+  MomentumArgs a{};
+  a.G = ch.Gt;
+  a.B = ch.Bt;
+  a.X = at<void>(ch, ch.L.X0);
+  a.ldx = g.ldx;
+  a.x_f32 = f32;
+  a.g_f32 = g_f32;
+  a.rows = g.rows;
+  a.cols = g.cols;
+  a.transposed = g.transposed;
+  a.cnt = ch.cnt;
+  a.mu = h.mu;
+  a.nesterov = h.nesterov;
+  a.partials = at<float>(ch, ch.L.partials);
+  a.nblk = ch.nblk;
+  a.aligned = ch.aligned;
+  const double bytes = static_cast<double>(g.rows) * g.cols * ch.cnt * ((g_f32 ? 4 : 2) + 8 + (f32 ? 4 : 2));
+  cudaError_t e = launch_k(KIND_EW, 0.0, bytes, s, [&] { return launch_momentum(a, s); });
+  if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "momentum kernel: %s", cudaGetErrorString(e));
+  e = launch_k(KIND_OTHER, 0.0, 0.0, s, [&] {
+    return launch_norm_finalize(at<float>(ch, ch.L.partials), ch.nblk, ch.cnt, h.eps, at<float>(ch, ch.L.s),
+                                at<float>(ch, ch.L.s2), s);
+  });
+  if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "norm finalize: %s", cudaGetErrorString(e));
+  return DMUON_OK;
+}
+
+// Newton-Schulz on X0 (unnormalised U, scale s folded into the first
+// products), finishing with `fin` (apply / out / store) on the result.
+int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int bn, const Hyper& h, const Epilogue& fin_in,
+           int cnt, cudaStream_t s) {
+  const Geo& g = *ch.g;
+  const int m = g.m, n = g.n;
+  const long long sx = g.x_elems(), sq = g.q_elems();
+  const float* sv = at<float>(ch, ch.L.s);
+  const float* s2v = at<float>(ch, ch.L.s2);
+  void* X0 = at<void>(ch, ch.L.X0);
+  Epilogue fin = fin_in;
+  int rc;
+  if (h.steps == 0) {  // O = X0 = s U; the kernel folds s in
+    fin.alpha = 1.f;
+    fin.alpha_vec = nullptr;
+    fin.beta = 0.f;
+    fin.C = nullptr;
+    cudaError_t e = launch_k(KIND_OTHER, 0.0, 0.0, s, [&] {
+      return launch_scale_epilogue(X0, g.ldx, f32, m, n, cnt, sv, fin, s);
+    });
+    if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "scale epilogue: %s", cudaGetErrorString(e));
+    return DMUON_OK;
+  }
+  if (variant == DMUON_VARIANT_GRAM) {
+    // Every m x m product takes its right operand as stored (MN-major B), not
+    // as the transpose of a matrix that is symmetric only up to rounding:
+    // multiplying by transposes feeds the rounding's antisymmetric part back
+    // into the recursion, where it grows from step to step (4e-2 instead of
+    // 1e-2 relative error after 5 steps at 96 x 200 in bf16).
+    void* A = at<void>(ch, ch.L.A);
+    void* P = at<void>(ch, ch.L.P);
+    void* T = at<void>(ch, ch.L.T);
+    void* Q[2] = {at<void>(ch, ch.L.Q0), at<void>(ch, ch.L.Q1)};
+    // G = s^2 U U^T  (A_0): both operands are rows of U (K-major)
+    rc = gemm(c, g, cnt, f32, bn, X0, g.ldx, sx, X0, g.ldx, sx, true, m, m, n, store_epi(A, g.ldm, sq, f32, 1.f, s2v), s);
+    if (rc) return rc;
+    int qi = 0;
+    for (int k = 0; k < h.steps; ++k) {
+      // P_k = c A_k^2 + b A_k + a I   (into Q[0] when k == 0: Q_1 = P_0)
+      void* Pk = (k == 0) ? Q[0] : P;
+      Epilogue ep = store_epi(Pk, g.ldm, sq, f32, h.c, nullptr);
+      ep.C = A;
+      ep.ldc = g.ldm;
+      ep.sc = sq;
+      ep.beta = h.b;
+      ep.diag = h.a;
+      rc = gemm(c, g, cnt, f32, bn, A, g.ldm, sq, A, g.ldm, sq, false, m, m, m, ep, s);
+      if (rc) return rc;
+      if (k > 0) {  // Q_{k+1} = P_k Q_k
+        rc = gemm(c, g, cnt, f32, bn, Pk, g.ldm, sq, Q[qi], g.ldm, sq, false, m, m, m,
+                  store_epi(Q[qi ^ 1], g.ldm, sq, f32, 1.f, nullptr), s);
+        if (rc) return rc;
+        qi ^= 1;
+      }
+      if (k < h.steps - 1) {  // A_{k+1} = P_k A_k P_k
+        rc = gemm(c, g, cnt, f32, bn, Pk, g.ldm, sq, A, g.ldm, sq, false, m, m, m,
+                  store_epi(T, g.ldm, sq, f32, 1.f, nullptr), s);
+        if (rc) return rc;
+        rc = gemm(c, g, cnt, f32, bn, T, g.ldm, sq, Pk, g.ldm, sq, false, m, m, m,
+                  store_epi(A, g.ldm, sq, f32, 1.f, nullptr), s);
+        if (rc) return rc;
+      }
+    }
+    // O = s * Q_K U
+    fin.alpha = 1.f;
+    fin.alpha_vec = sv;
+    fin.beta = 0.f;
+    fin.C = nullptr;
+    return gemm(c, g, cnt, f32, bn, Q[qi], g.ldm, sq, X0, g.ldx, sx, false, m, n, m, fin, s);
+  }
+  // ---------------- direct form
+  void* A = at<void>(ch, ch.L.A);
+  void* Bm = at<void>(ch, ch.L.Bm);
+  void* bufs[2] = {at<void>(ch, ch.L.Xp), at<void>(ch, ch.L.Xq)};
+  void* cur = X0;
+  for (int k = 0; k < h.steps; ++k) {
+    const bool first = (k == 0);
+    const bool last = (k == h.steps - 1);
+    // A = X X^T  (s^2 folded in on the first step)
+    rc = gemm(c, g, cnt, f32, bn, cur, g.ldx, sx, cur, g.ldx, sx, true, m, m, n,
+              store_epi(A, g.ldm, sq, f32, 1.f, first ? s2v : nullptr), s);
+    if (rc) return rc;
+    // Bm = c A A + b A   (right operand as stored, see the Gram form)
+    Epilogue ep = store_epi(Bm, g.ldm, sq, f32, h.c, nullptr);
+    ep.C = A;
+    ep.ldc = g.ldm;
+    ep.sc = sq;
+    ep.beta = h.b;
+    rc = gemm(c, g, cnt, f32, bn, A, g.ldm, sq, A, g.ldm, sq, false, m, m, m, ep, s);
+    if (rc) return rc;
+    // X' = Bm X + a X   (times s on the first step)
+    void* nxt = bufs[k & 1];
+    Epilogue eu = last ? fin : store_epi(nxt, g.ldx, sx, f32, 1.f, nullptr);
+    eu.alpha = 1.f;
+    eu.alpha_vec = first ? sv : nullptr;
+    eu.beta = h.a;
+    eu.beta_vec = first ? sv : nullptr;
+    eu.C = cur;
+    eu.ldc = g.ldx;
+    eu.sc = sx;
+    eu.c_f32 = f32;
+    rc = gemm(c, g, cnt, f32, bn, Bm, g.ldm, sq, cur, g.ldx, sx, false, m, n, m, eu, s);
+    if (rc) return rc;
+    cur = nxt;
+  }
+  return DMUON_OK;
+}
+
+// ------------------------------------------------------------------ step
+struct Group {
+  long long rows, cols;
+  std::vector<int> idx;
+  Plan plan;
+  int chunk;
+};
+
+struct Request {
+  void* const* params;
+  const void* const* grads;
+  void* const* moms;
+  float* const* out;  // dmuon_compute_update
+  const int64_t* shapes;
+  int count;
+  Hyper h;
+  dmuon_options o;
+  cudaStream_t s;
+};
+
+int validate(const Request& r) {
+  if (r.count < 0) return fail(DMUON_ERR_INVALID, "count < 0");
+  if (r.count == 0) return DMUON_OK;
+  if (!r.grads || !r.moms || !r.shapes || (!r.params && !r.out))
+    return fail(DMUON_ERR_INVALID, "null pointer array");
+  if (r.h.steps < 0 || r.h.steps > 16) return fail(DMUON_ERR_INVALID, "ns_steps %d outside [0, 16]", r.h.steps);
+  const float hs[] = {r.h.lr, r.h.wd, r.h.mu, r.h.eps, r.h.a, r.h.b, r.h.c};
+  for (float v : hs)
+    if (!std::isfinite(v)) return fail(DMUON_ERR_INVALID, "non-finite hyperparameter");
+  if (r.h.eps < 0.f) return fail(DMUON_ERR_INVALID, "eps < 0");
+  const dmuon_options& o = r.o;
+  if (o.mom_dtype != DMUON_F32) return fail(DMUON_ERR_DTYPE, "momentum dtype must be F32");
+  if (!((o.param_dtype == DMUON_BF16 && o.grad_dtype == DMUON_BF16) ||
+        (o.param_dtype == DMUON_F32 && o.grad_dtype == DMUON_F32)))
+    return fail(DMUON_ERR_DTYPE, "param/grad dtypes must both be BF16 or both F32");
+  if (o.variant < 0 || o.variant > 3) return fail(DMUON_ERR_INVALID, "unknown variant %d", o.variant);
+  for (int i = 0; i < r.count; ++i) {
+    const int64_t rr = r.shapes[2 * i], cc = r.shapes[2 * i + 1];
+    if (rr <= 0 || cc <= 0) return fail(DMUON_ERR_INVALID, "matrix %d has shape %lld x %lld", i, (long long)rr, (long long)cc);
+    if (rr > (1 << 20) || cc > (1 << 20) || rr * cc > (1LL << 31))
+      return fail(DMUON_ERR_INVALID, "matrix %d shape %lld x %lld too large", i, (long long)rr, (long long)cc);
+    if (!r.grads[i] || !r.moms[i] || (r.params && !r.params[i]) || (r.out && !r.out[i]))
+      return fail(DMUON_ERR_INVALID, "null pointer for matrix %d", i);
+  }
+  return DMUON_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int forced_bn() {
+  const char* b = getenv("DMUON_BN");
+  if (b) {
+    int v = atoi(b);
+    if (v == 128 || v == 256) return v;
+  }
+  return 0;
+}
+
+double gate_tol() {
+  const char* g = getenv("DMUON_GATE");
+  return g ? atof(g) : 2e-2;
+}
+
+int upload_tables(DeviceCtx& c, const std::vector<void*>& host, void* dev, cudaStream_t s) {
+  const size_t bytes = host.size() * sizeof(void*);
+  if (bytes == 0) return DMUON_OK;
+  const int slot = c.pin_next;
+  if (c.pin_used[slot]) CUDA_TRY(cudaEventSynchronize(c.pin_ev[slot]));
+  if (c.pin_cap[slot] < bytes) {
+    if (c.pin[slot]) CUDA_TRY(cudaFreeHost(c.pin[slot]));
+    c.pin[slot] = nullptr;
+    size_t cap = std::max<size_t>(bytes, 64 << 10);
+    CUDA_TRY(cudaHostAlloc(&c.pin[slot], cap, cudaHostAllocDefault));
+    c.pin_cap[slot] = cap;
+  }
+  memcpy(c.pin[slot], host.data(), bytes);
+  CUDA_TRY(cudaMemcpyAsync(dev, c.pin[slot], bytes, cudaMemcpyHostToDevice, s));
+  CUDA_TRY(cudaEventRecord(c.pin_ev[slot], s));
+  c.pin_used[slot] = true;
+  c.pin_next ^= 1;
+  return DMUON_OK;
+}
+
+Epilogue final_epilogue(const Request& r, const Geo& g, const Chunk& ch, bool f32) {
+  Epilogue e{};
+  e.transposed = g.transposed;
+  e.ldw = g.cols;
+  e.w_f32 = f32;
+  if (r.out) {
+    e.mode = EPI_OUT;
+    e.Out = ch.Ot;
+  } else {
+    e.mode = EPI_APPLY;
+    e.W = ch.Wt;
+    e.decay = 1.f - r.h.lr * r.h.wd;
+    e.lr_scale = r.h.lr * 0.2f * std::sqrt(static_cast<float>(std::max(g.rows, g.cols)));
+  }
+  return e;
+}
+
+int time_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int bn, const Hyper& h, const Epilogue& fin,
+            int cnt, cudaStream_t s, float* ms) {
+  CUDA_TRY(cudaEventRecord(c.tune_a, s));
+  int rc = run_ns(c, ch, f32, variant, bn, h, fin, cnt, s);
+  if (rc) return rc;
+  CUDA_TRY(cudaEventRecord(c.tune_b, s));
+  CUDA_TRY(cudaEventSynchronize(c.tune_b));
+  CUDA_TRY(cudaEventElapsedTime(ms, c.tune_a, c.tune_b));
+  if (*c.err_host) return fail(DMUON_ERR_DEVICE_TIMEOUT, "device wait timed out during autotune");
+  return DMUON_OK;
+}
+
+// Chooses the plan for a group by timing candidates on the chunk's own data
+// (after the momentum kernel produced X0).  Candidates write their result
+// into scratch (Xq region reused as the output), never into the caller's
+// buffers.  Direct form with bn 256 is the accuracy reference of the gate.
+int autotune(DeviceCtx& c, const Chunk& ch, bool f32, const Hyper& h, int forced_variant, Plan* plan,
+             cudaStream_t s) {
+  const Geo& g = *ch.g;
+  std::vector<std::pair<int, int>> cands;  // (variant, bn)
+  const int fbn = forced_bn();
+  std::vector<int> bns;
+  if (f32)
+    bns = {0};
+  else if (fbn)
+    bns = {fbn};
+  else
+    bns = {256, 128};
+  std::vector<int> vars;
+  if (forced_variant == DMUON_VARIANT_DIRECT || forced_variant == DMUON_VARIANT_GRAM)
+    vars = {forced_variant};
+  else {
+    vars = {DMUON_VARIANT_DIRECT};
+    if (g.n * 4 >= g.m * 5 && h.steps > 0) vars.push_back(DMUON_VARIANT_GRAM);  // n >= 1.25 m
+  }
+  for (int v : vars)
+    for (int b : bns) cands.push_back({v, b});
+  if (h.steps == 0) cands = {{DMUON_VARIANT_DIRECT, bns[0]}};
+
+  // Output of each candidate: reuse the Xp region for the reference and a
+  // second region (Xq) for the challenger; direct ping-pongs Xp/Xq itself,
+  // so candidates store their final result into the P/Q regions' space only
+  // when it fits.  Simplest safe choice: store the final result in X-sized
+  // scratch appended after the layout (`out` below).
+  const int probe = ch.cnt;
+  uint8_t* outbuf = ch.base + ch.L.total;  // two X-sized slots reserved by the caller
+  const size_t xb = align256(static_cast<size_t>(probe) * g.x_elems() * g.esz);
+  void* ref_out = outbuf;
+  void* cand_out = outbuf + xb;
+  double* dacc = reinterpret_cast<double*>(outbuf + 2 * xb);
+
+  float best = 1e30f;
+  Plan bestp;
+  bool have_ref = false;
+  for (auto [v, bn] : cands) {
+    const bool is_ref = !have_ref;
+    void* dst = is_ref ? ref_out : cand_out;
+    Epilogue fin = store_epi(dst, g.ldx, g.x_elems(), f32, 1.f, nullptr);
+    float ms = 0.f;
+    // warm once (first launch of a kernel instance loads the module), then time
+    int rc = run_ns(c, ch, f32, v, bn == 0 ? 256 : bn, h, fin, probe, s);
+    if (rc) return rc;
+    rc = time_ns(c, ch, f32, v, bn == 0 ? 256 : bn, h, fin, probe, s, &ms);
+    if (rc) return rc;
+    bool pass = true;
+    double relerr = 0.0;
+    if (!is_ref) {
+      CUDA_TRY(cudaMemsetAsync(dacc, 0, 2 * sizeof(double), s));
+      cudaError_t e = launch_diff_norms(cand_out, ref_out, g.ldx, g.m, g.n, probe, f32, dacc, s);
+      if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "diff norms: %s", cudaGetErrorString(e));
+      double hacc[2];
+      CUDA_TRY(cudaMemcpyAsync(hacc, dacc, sizeof(hacc), cudaMemcpyDeviceToHost, s));
+      CUDA_TRY(cudaStreamSynchronize(s));
+      relerr = hacc[1] > 0 ? std::sqrt(hacc[0] / hacc[1]) : std::sqrt(hacc[0]);
+      pass = relerr <= gate_tol();
+    }
+    if (trace_on())
+      fprintf(stderr, "[dmuon] tune %dx%d cnt=%d variant=%d bn=%d: %.3f ms%s gate=%.2e %s\n", g.rows, g.cols, probe, v,
+              bn, ms, is_ref ? " (reference)" : "", relerr, pass ? "pass" : "REJECT");
+    have_ref = true;
+    if (pass && ms < best) {
+      best = ms;
+      bestp.variant = v;
+      bestp.bn = bn == 0 ? 256 : bn;
+      bestp.cost_ms = ms;
+    }
+  }
+  *plan = bestp;
+  return DMUON_OK;
+}
+
+
+int run_step(Request& r) {
+  int rc = validate(r);
+  if (rc || r.count == 0) return rc;
+  DeviceCtx* cp = nullptr;
+  rc = get_ctx(&cp);
+  if (rc) return rc;
+  DeviceCtx& c = *cp;
+  std::lock_guard<std::mutex> lk(c.mu);
+  if (*c.err_host) {
+    *c.err_host = 0;
+    return fail(DMUON_ERR_DEVICE_TIMEOUT, "a previous launch on this device timed out on a device-side wait");
+  }
+  const bool f32 = r.o.param_dtype == DMUON_F32;
+  const bool g_f32 = r.o.grad_dtype == DMUON_F32;
+
+  // group by shape, in order of first appearance
+  std::vector<Group> groups;
+  {
+    std::map<std::pair<long long, long long>, int> gi;
+    for (int i = 0; i < r.count; ++i) {
+      auto key = std::make_pair(static_cast<long long>(r.shapes[2 * i]), static_cast<long long>(r.shapes[2 * i + 1]));
+      auto it = gi.find(key);
+      if (it == gi.end()) {
+        it = gi.emplace(key, static_cast<int>(groups.size())).first;
+        groups.push_back(Group{key.first, key.second, {}, Plan{}, 0});
+      }
+      groups[it->second].idx.push_back(i);
+    }
+  }
+  // plans: cache lookup; misses are tuned on this call's data below
+  std::vector<Geo> geos(groups.size());
+  std::vector<bool> miss(groups.size(), false);
+  size_t ws_need = 0;
+  for (size_t k = 0; k < groups.size(); ++k) {
+    Group& gr = groups[k];
+    geos[k] = make_geo(gr.rows, gr.cols, f32);
+    gr.chunk = chunk_size(geos[k], static_cast<int>(gr.idx.size()));
+    Key key{gr.rows, gr.cols, f32 ? 1 : 0, r.h.steps, gr.chunk};
+    {
+      std::lock_guard<std::mutex> lk2(g_cache_mu);
+      auto it = g_cache.find(key);
+      if (it != g_cache.end() && (r.o.variant == DMUON_VARIANT_AUTO || it->second.variant == r.o.variant)) {
+        gr.plan = it->second;
+      } else {
+        miss[k] = true;
+      }
+    }
+    const int nblk = momentum_partials(geos[k].rows, geos[k].cols, gr.chunk, c.num_sms);
+    Layout L = make_layout(geos[k], gr.chunk, nblk);
+    size_t need = L.total;
+    if (miss[k]) need += 2 * align256(static_cast<size_t>(gr.chunk) * geos[k].x_elems() * geos[k].esz) + 256;
+    ws_need = std::max(ws_need, need);
+  }
+  // device pointer tables: 4 arrays of count pointers, after the chunk scratch
+  const size_t tables_off = align256(ws_need);
+  const size_t total_ws = tables_off + align256(4 * sizeof(void*) * static_cast<size_t>(r.count));
+  rc = ensure_ws(c, total_ws, r.s);
+  if (rc) return rc;
+
+  // order GPU work after the previous call's (it may be on another stream)
+  if (c.has_last) CUDA_TRY(cudaStreamWaitEvent(r.s, c.last_done, 0));
+
+  // pointer tables, grouped: for group k, its matrices are contiguous
+  std::vector<void*> host(4 * static_cast<size_t>(r.count));
+  std::vector<int> gstart(groups.size());
+  {
+    int pos = 0;
+    for (size_t k = 0; k < groups.size(); ++k) {
+      gstart[k] = pos;
+      for (int i : groups[k].idx) {
+        host[pos] = const_cast<void*>(r.grads[i]);
+        host[r.count + pos] = r.moms[i];
+        host[2 * r.count + pos] = r.params ? r.params[i] : nullptr;
+        host[3 * r.count + pos] = r.out ? static_cast<void*>(r.out[i]) : nullptr;
+        ++pos;
+      }
+    }
+  }
+  uint8_t* ws = static_cast<uint8_t*>(c.ws);
+  void** dtab = reinterpret_cast<void**>(ws + tables_off);
+  rc = upload_tables(c, host, dtab, r.s);
+  if (rc) return rc;
+
+  // issue order: tuned groups first (they synchronise), then by cost
+  std::vector<int> order(groups.size());
+  for (size_t k = 0; k < order.size(); ++k) order[k] = static_cast<int>(k);
+  std::stable_sort(order.begin(), order.end(), [&](int x, int y) {
+    if (miss[x] != miss[y]) return static_cast<bool>(miss[x]);
+    const double cx = groups[x].plan.cost_ms * ((groups[x].idx.size() + groups[x].chunk - 1) / groups[x].chunk);
+    const double cy = groups[y].plan.cost_ms * ((groups[y].idx.size() + groups[y].chunk - 1) / groups[y].chunk);
+    return cx > cy;
+  });
+
+  for (int k : order) {
+    Group& gr = groups[k];
+    const Geo& g = geos[k];
+    const int total = static_cast<int>(gr.idx.size());
+    for (int c0 = 0; c0 < total; c0 += gr.chunk) {
+      Chunk ch;
+      ch.g = &g;
+      ch.cnt = std::min(gr.chunk, total - c0);
+      ch.base = ws;
+      ch.nblk = momentum_partials(g.rows, g.cols, gr.chunk, c.num_sms);
+      ch.L = make_layout(g, gr.chunk, ch.nblk);
+      const int p = gstart[k] + c0;
+      ch.Gt = dtab + p;
+      ch.Bt = dtab + r.count + p;
+      ch.Wt = dtab + 2 * r.count + p;
+      ch.Ot = reinterpret_cast<float* const*>(dtab + 3 * r.count + p);
+      ch.aligned = 1;
+      for (int q = 0; q < ch.cnt; ++q) {
+        const int i = gr.idx[c0 + q];
+        if (!aligned16(r.grads[i]) || !aligned16(r.moms[i])) ch.aligned = 0;
+      }
+      rc = run_momentum(c, ch, f32, g_f32, r.h, r.s);
+      if (rc) return rc;
+      if (miss[k] && c0 == 0) {
+        Plan pl;
+        rc = autotune(c, ch, f32, r.h, r.o.variant, &pl, r.s);
+        if (rc) return rc;
+        gr.plan = pl;
+        Key key{gr.rows, gr.cols, f32 ? 1 : 0, r.h.steps, gr.chunk};
+        std::lock_guard<std::mutex> lk2(g_cache_mu);
+        if (r.o.variant == DMUON_VARIANT_AUTO || !g_cache.count(key)) g_cache[key] = pl;
+      }
+      Epilogue fin = final_epilogue(r, g, ch, f32);
+      rc = run_ns(c, ch, f32, gr.plan.variant, gr.plan.bn, r.h, fin, ch.cnt, r.s);
+      if (rc) return rc;
+    }
+    if (trace_on())
+      fprintf(stderr, "[dmuon] group %lldx%lld x%d: variant=%d bn=%d chunk=%d cost=%.3f ms\n", gr.rows, gr.cols, total,
+              gr.plan.variant, gr.plan.bn, gr.chunk, gr.plan.cost_ms);
+  }
+  CUDA_TRY(cudaEventRecord(c.last_done, r.s));
+  c.has_last = true;
+  return DMUON_OK;
+}
+
+Hyper hyper_from(float lr, float wd, float mu, int steps, const dmuon_options& o) {
+  Hyper h;
+  h.mu = mu;
+  h.lr = lr;
+  h.wd = wd;
+  h.eps = o.eps;
+  h.a = o.ns_a;
+  h.b = o.ns_b;
+  h.c = o.ns_c;
+  h.steps = steps;
+  h.nesterov = o.nesterov;
+  return h;
+}
+
+}  // namespace
+}  // namespace dmuon
+
+using namespace dmuon;
+
+extern "C" {
+
+void dmuon_options_init(dmuon_options* o) {
+  if (!o) return;
+  o->param_dtype = DMUON_BF16;
+  o->grad_dtype = DMUON_BF16;
+  o->mom_dtype = DMUON_F32;
+  o->eps = 1e-7f;
+  o->nesterov = 1;
+  o->variant = DMUON_VARIANT_AUTO;
+  o->ns_a = 3.4445f;
+  o->ns_b = -4.7750f;
+  o->ns_c = 2.0315f;
+}
+
+int dmuon_step_ex(void* const* params, const void* const* grads, void* const* momenta, const int64_t* shapes,
+                  int count, float lr, float wd, float mu, int ns_steps, const dmuon_options* opts, void* stream) {
+  t_err.clear();
+  dmuon_options o;
+  dmuon_options_init(&o);
+  if (opts) o = *opts;
+  if (!params && count > 0) return fail(DMUON_ERR_INVALID, "params is NULL");
+  Request r{params, grads, momenta, nullptr, shapes, count, hyper_from(lr, wd, mu, ns_steps, o), o,
+            static_cast<cudaStream_t>(stream)};
+  return run_step(r);
+}
+
+int dmuon_step(void* const* params, const void* const* grads, void* const* momenta, const int64_t* shapes, int count,
+               float lr, float wd, float mu, int ns_steps, void* stream) {
+  return dmuon_step_ex(params, grads, momenta, shapes, count, lr, wd, mu, ns_steps, nullptr, stream);
+}
+
+int dmuon_compute_update(const void* const* grads, void* const* momenta, const int64_t* shapes, int count, float mu,
+                         int ns_steps, const dmuon_options* opts, float* const* out, void* stream) {
+  t_err.clear();
+  dmuon_options o;
+  dmuon_options_init(&o);
+  if (opts) o = *opts;
+  if (!out && count > 0) return fail(DMUON_ERR_INVALID, "out is NULL");
+  Request r{nullptr, grads, momenta, out, shapes, count, hyper_from(0.f, 0.f, mu, ns_steps, o), o,
+            static_cast<cudaStream_t>(stream)};
+  return run_step(r);
+}
+
+int dmuon_gemm_bf16(const void* A, int64_t lda, int64_t sa, const void* B, int64_t ldb, int64_t sb, int b_kmajor,
+                    const void* C, int64_t ldc, int64_t sc, void* D, int64_t ldd, int64_t sd, int M, int N, int K,
+                    int batch, float alpha, float beta, int bn, void* stream) {
+  t_err.clear();
+  if (!A || !B || !D) return fail(DMUON_ERR_INVALID, "null operand");
+  if (M <= 0 || N <= 0 || K <= 0 || batch <= 0) return fail(DMUON_ERR_INVALID, "bad GEMM size");
+  if ((lda | ldb | ldd | sa | sb | sd) & 7 || (C && ((ldc | sc) & 7)))
+    return fail(DMUON_ERR_INVALID, "leading dims / batch strides must be multiples of 8");
+  if (lda < K || ldd < N || (b_kmajor ? ldb < K : ldb < N) || (C && ldc < N))
+    return fail(DMUON_ERR_INVALID, "leading dim smaller than the row");
+  if (bn != 0 && bn != 128 && bn != 256) return fail(DMUON_ERR_INVALID, "bn must be 0, 128 or 256");
+  DeviceCtx* cp = nullptr;
+  int rc = get_ctx(&cp);
+  if (rc) return rc;
+  Epilogue e{};
+  e.mode = EPI_STORE;
+  e.alpha = alpha;
+  e.beta = beta;
+  e.C = C;
+  e.ldc = ldc;
+  e.sc = sc;
+  e.D = D;
+  e.ldd = ldd;
+  e.sd = sd;
+  TcGemm t{A, lda, sa, B, ldb, sb, b_kmajor != 0, M, N, K, batch, bn == 0 ? 256 : bn, e};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t err = launch_k(KIND_TC_GEMM, 2.0 * M * N * static_cast<double>(K) * batch, 0.0, s,
+                             [&] { return launch_tc_gemm(t, s, cp->err_dev, cp->num_sms); });
+  if (err != cudaSuccess) return fail(DMUON_ERR_CUDA, "gemm launch: %s", cudaGetErrorString(err));
+  return DMUON_OK;
+}
+
+int dmuon_cache_save(const char* path) {
+  t_err.clear();
+  if (!path) return fail(DMUON_ERR_INVALID, "null path");
+  DeviceCtx* cp = nullptr;
+  int rc = get_ctx(&cp);
+  if (rc) return rc;
+  FILE* f = fopen(path, "w");
+  if (!f) return fail(DMUON_ERR_INVALID, "cannot open %s", path);
+  std::string gpu = cp->name;
+  for (char& ch : gpu)
+    if (ch == ' ') ch = '_';
+  fprintf(f, "dmuon-cache %d %s %d\n", DMUON_VERSION, gpu.c_str(), cp->num_sms);
+  std::lock_guard<std::mutex> lk(g_cache_mu);
+  for (auto& kv : g_cache)
+    fprintf(f, "%lld %lld %d %d %d %d %d %.6f\n", kv.first.rows, kv.first.cols, kv.first.f32, kv.first.steps,
+            kv.first.cnt, kv.second.variant, kv.second.bn, kv.second.cost_ms);
+  fclose(f);
+  return DMUON_OK;
+}
+
+int dmuon_cache_load(const char* path) {
+  t_err.clear();
+  if (!path) return fail(DMUON_ERR_INVALID, "null path");
+  DeviceCtx* cp = nullptr;
+  int rc = get_ctx(&cp);
+  if (rc) return rc;
+  FILE* f = fopen(path, "r");
+  if (!f) return fail(DMUON_ERR_INVALID, "cannot open %s", path);
+  int ver = 0, sms = 0;
+  char gpu[256] = {0};
+  if (fscanf(f, "dmuon-cache %d %255s %d", &ver, gpu, &sms) != 3) {
+    fclose(f);
+    return fail(DMUON_ERR_INVALID, "%s: not a dmuon cache file", path);
+  }
+  std::string mine = cp->name;
+  for (char& ch : mine)
+    if (ch == ' ') ch = '_';
+  if (ver != DMUON_VERSION || mine != gpu || sms != cp->num_sms) {
+    fclose(f);
+    return fail(DMUON_ERR_INVALID, "%s was tuned for %s (%d SMs, v%d), not this GPU", path, gpu, sms, ver);
+  }
+  std::map<Key, Plan> loaded;
+  long long rr, cc;
+  int f32, steps, cnt, var, bn;
+  double cost;
+  while (fscanf(f, "%lld %lld %d %d %d %d %d %lf", &rr, &cc, &f32, &steps, &cnt, &var, &bn, &cost) == 8) {
+    if (rr <= 0 || cc <= 0 || cnt <= 0 || (var != 1 && var != 2) || (bn != 128 && bn != 256)) {
+      fclose(f);
+      return fail(DMUON_ERR_INVALID, "%s: malformed entry", path);
+    }
+    Plan p;
+    p.variant = var;
+    p.bn = bn;
+    p.cost_ms = cost;
+    loaded[Key{rr, cc, f32, steps, cnt}] = p;
+  }
+  fclose(f);
+  std::lock_guard<std::mutex> lk(g_cache_mu);
+  for (auto& kv : loaded) g_cache[kv.first] = kv.second;
+  return DMUON_OK;
+}
+
+void dmuon_cache_clear(void) {
+  std::lock_guard<std::mutex> lk(g_cache_mu);
+  g_cache.clear();
+}
+
+int dmuon_cache_size(void) {
+  std::lock_guard<std::mutex> lk(g_cache_mu);
+  return static_cast<int>(g_cache.size());
+}
+
+int dmuon_cache_entry(int i, char* buf, size_t len) {
+  std::lock_guard<std::mutex> lk(g_cache_mu);
+  if (i < 0 || i >= static_cast<int>(g_cache.size()) || !buf || len == 0)
+    return fail(DMUON_ERR_INVALID, "bad cache index");
+  auto it = g_cache.begin();
+  std::advance(it, i);
+  snprintf(buf, len, "%lld %lld %s %d %s %d %d %.4f", it->first.rows, it->first.cols, it->first.f32 ? "f32" : "bf16",
+           it->first.steps, it->second.variant == DMUON_VARIANT_GRAM ? "gram" : "direct", it->second.bn, it->first.cnt,
+           it->second.cost_ms);
+  return DMUON_OK;
+}
+
+int dmuon_set_workspace(void* dev_ptr, size_t bytes) {
+  t_err.clear();
+  if (dev_ptr && (reinterpret_cast<uintptr_t>(dev_ptr) & 255))
+    return fail(DMUON_ERR_INVALID, "workspace must be 256-byte aligned");
+  g_ext_ptr = bytes ? dev_ptr : nullptr;
+  g_ext_bytes = dev_ptr ? bytes : 0;
+  return DMUON_OK;
+}
+
+int dmuon_workspace_size(const int64_t* shapes, int count, int param_dtype, size_t* bytes) {
+  t_err.clear();
+  if (!bytes || (count > 0 && !shapes) || count < 0) return fail(DMUON_ERR_INVALID, "bad arguments");
+  const bool f32 = param_dtype == DMUON_F32;
+  std::map<std::pair<long long, long long>, int> counts;
+  for (int i = 0; i < count; ++i) {
+    if (shapes[2 * i] <= 0 || shapes[2 * i + 1] <= 0) return fail(DMUON_ERR_INVALID, "bad shape");
+    counts[{shapes[2 * i], shapes[2 * i + 1]}]++;
+  }
+  size_t need = 0;
+  for (auto& kv : counts) {
+    Geo g = make_geo(kv.first.first, kv.first.second, f32);
+    int ch = chunk_size(g, kv.second);
+    Layout L = make_layout(g, ch, momentum_partials(g.rows, g.cols, ch, 148));
+    need = std::max(need, L.total + 2 * align256(static_cast<size_t>(ch) * g.x_elems() * g.esz) + 256);
+  }
+  *bytes = align256(need) + align256(4 * sizeof(void*) * static_cast<size_t>(count));
+  return DMUON_OK;
+}
+
+void dmuon_timing_enable(int enable) { g_timing.store(enable ? 1 : 0); }
+
+void dmuon_timing_reset(void) {
+  std::lock_guard<std::mutex> lk(g_tmu);
+  for (auto& t : g_timed) {
+    g_event_pool.push_back(t.a);
+    g_event_pool.push_back(t.b);
+  }
+  g_timed.clear();
+}
+
+int dmuon_timing_get(int kind, int64_t* launches, double* ms, double* flops, double* bytes) {
+  std::lock_guard<std::mutex> lk(g_tmu);
+  int64_t n = 0;
+  double t = 0, f = 0, b = 0;
+  for (auto& x : g_timed) {
+    if (x.kind != kind) continue;
+    cudaError_t e = cudaEventSynchronize(x.b);
+    if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "timing event: %s", cudaGetErrorString(e));
+    float d = 0.f;
+    cudaEventElapsedTime(&d, x.a, x.b);
+    ++n;
+    t += d;
+    f += x.flops;
+    b += x.bytes;
+  }
+  if (launches) *launches = n;
+  if (ms) *ms = t;
+  if (flops) *flops = f;
+  if (bytes) *bytes = b;
+  return DMUON_OK;
+}
+
+int64_t dmuon_launch_count(void) { return g_launches.load(); }
+
+const char* dmuon_last_error(void) { return t_err.c_str(); }
+
+int dmuon_version(void) { return DMUON_VERSION; }
+
+}  // extern "C"

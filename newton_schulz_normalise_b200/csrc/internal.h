@@ -1,0 +1,76 @@
+// internal.h -- launchers shared by the library's host code (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace dmuon {
+
+// Batched GEMM on the tensor cores:  D[l] = epi(A[l] * op(B[l]))
+//   A  bf16, M x K, K contiguous (row stride lda, batch stride sa, elements)
+//   B  bf16, b_kmajor ? N x K (K contiguous) : K x N (N contiguous)
+struct TcGemm {
+  const void* A;
+  long long lda, sa;
+  const void* B;
+  long long ldb, sb;
+  bool b_kmajor;
+  int M, N, K, batch;
+  int bn;  // tile width: 128 or 256
+  Epilogue epi;
+};
+
+// Same contract in fp32 on the CUDA cores (fp32 path; any leading dims).
+struct SimtGemm {
+  const float* A;
+  long long lda, sa;
+  const float* B;
+  long long ldb, sb;
+  bool b_kmajor;
+  int M, N, K, batch;
+  Epilogue epi;
+};
+
+// Kernel classes for timing (dmuon_timing_get).
+enum KernelKind { KIND_TC_GEMM = 0, KIND_EW = 1, KIND_SIMT_GEMM = 2, KIND_OTHER = 3, KIND_COUNT = 4 };
+
+cudaError_t launch_tc_gemm(const TcGemm& g, cudaStream_t s, int* dev_err, int num_sms);
+cudaError_t launch_simt_gemm(const SimtGemm& g, cudaStream_t s);
+
+// Momentum + Nesterov + per-matrix sum of squares (partials), writing the
+// wide-orientation iterate X (bf16 or fp32) for `cnt` same-shape matrices.
+struct MomentumArgs {
+  const void* const* G;  // device table of cnt pointers
+  void* const* B;        // device table of cnt pointers (fp32, updated in place)
+  void* X;               // [cnt][m][ldx] wide orientation
+  long long ldx;
+  int x_f32, g_f32;
+  int rows, cols;        // stored shape
+  int transposed;        // rows > cols
+  int cnt;
+  float mu;
+  int nesterov;
+  float* partials;       // [cnt][nblk]
+  int nblk;              // partial slots per matrix
+  int aligned;           // every G/B base 16-byte aligned (vector path allowed)
+};
+cudaError_t launch_momentum(const MomentumArgs& a, cudaStream_t s);
+// Number of partial slots launch_momentum uses for this shape.
+int momentum_partials(int rows, int cols, int cnt, int num_sms);
+
+// s[l] = 1 / (sqrt(sum partials[l][:]) + eps),  s2[l] = s[l]^2.
+cudaError_t launch_norm_finalize(const float* partials, int nblk, int cnt, float eps, float* s, float* s2,
+                                 cudaStream_t st);
+
+// O = s[l] * X (zero Newton-Schulz steps) through the epilogue (apply / out).
+cudaError_t launch_scale_epilogue(const void* X, long long ldx, int x_f32, int m, int n, int cnt,
+                                  const float* s, const Epilogue& epi, cudaStream_t st);
+
+// Relative Frobenius distance helper for the autotuner's accuracy gate:
+// acc[0] += sum (x - y)^2, acc[1] += sum y^2 over cnt matrices m x n (ld).
+cudaError_t launch_diff_norms(const void* X, const void* Y, long long ld, int m, int n, int cnt, int is_f32,
+                              double* acc, cudaStream_t st);
+
+}  // namespace dmuon

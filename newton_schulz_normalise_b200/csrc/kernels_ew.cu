@@ -1,0 +1,277 @@
+// kernels_ew.cu -- the HBM-bound elementwise stages of the Muon step.
+//
+// launch_momentum: one pass over G and B per matrix:
+//     B' = mu*B + G  (written back, fp32),  U = G + mu*B' (or B'),
+//     X  = U (or U^T for tall matrices) written as the bf16/fp32 iterate,
+//     per-block partial sums of U^2 for the Frobenius norm.
+//   12 bytes per element for bf16 G / fp32 B / bf16 X: read G (2), read and
+//   write B (8), write X (2).  128-bit loads/stores on the aligned path; tall
+//   matrices go through a 64x64 shared-memory transpose so both the reads and
+//   the writes stay coalesced.
+// launch_norm_finalize: s = 1/(||U||_F + eps) from the partials, in a fixed
+//   order (deterministic).
+// launch_scale_epilogue: O = s*X for zero Newton-Schulz steps.
+// launch_diff_norms: ||X - Y||^2 and ||Y||^2 for the autotuner's gate.
+#include "internal.h"
+
+namespace dmuon {
+
+namespace {
+
+constexpr int EW_THREADS = 256;
+constexpr int VEC = 8;
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  float r = 0.f;
+  if (threadIdx.x < 32) {
+    r = lane < static_cast<int>(blockDim.x >> 5) ? red[lane] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+  }
+  return r;  // valid in thread 0
+}
+
+__device__ __forceinline__ void load8(const void* p, long long i, int is_f32, float (&g)[8]) {
+  if (is_f32) {
+    const float4* q = reinterpret_cast<const float4*>(static_cast<const float*>(p) + i);
+    float4 a = __ldcs(q), b = __ldcs(q + 1);
+    g[0] = a.x; g[1] = a.y; g[2] = a.z; g[3] = a.w; g[4] = b.x; g[5] = b.y; g[6] = b.z; g[7] = b.w;
+  } else {
+    uint4 u = __ldcs(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p) + i));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      float2 f = __bfloat1622float2(h[t]);
+      g[2 * t] = f.x;
+      g[2 * t + 1] = f.y;
+    }
+  }
+}
+
+__device__ __forceinline__ void store8(void* p, long long i, int is_f32, const float (&x)[8]) {
+  if (is_f32) {
+    float4* q = reinterpret_cast<float4*>(static_cast<float*>(p) + i);
+    q[0] = make_float4(x[0], x[1], x[2], x[3]);
+    q[1] = make_float4(x[4], x[5], x[6], x[7]);
+  } else {
+    uint4 u;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) h[t] = __floats2bfloat162_rn(x[2 * t], x[2 * t + 1]);
+    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p) + i) = u;
+  }
+}
+
+// Wide (rows <= cols) matrices: X has the stored layout (row stride ldx).
+__global__ void __launch_bounds__(EW_THREADS) momentum_wide_kernel(const MomentumArgs a, int vec_ok) {
+  __shared__ float red[EW_THREADS / 32];
+  const int l = blockIdx.y;
+  const void* G = a.G[l];
+  float* B = static_cast<float*>(a.B[l]);
+  const long long xoff = static_cast<long long>(l) * a.rows * a.ldx;
+  const long long numel = static_cast<long long>(a.rows) * a.cols;
+  const float mu = a.mu;
+  float ss = 0.f;
+  if (vec_ok) {
+    // cols % 8 == 0 and every base 16/32-byte aligned: ldx == cols.
+    const long long nvec = numel / VEC;
+    for (long long v = static_cast<long long>(blockIdx.x) * EW_THREADS + threadIdx.x; v < nvec;
+         v += static_cast<long long>(gridDim.x) * EW_THREADS) {
+      const long long i = v * VEC;
+      float g[8], b[8], u[8];
+      load8(G, i, a.g_f32, g);
+      load8(B, i, 1, b);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        b[t] = fmaf(mu, b[t], g[t]);
+        u[t] = a.nesterov ? fmaf(mu, b[t], g[t]) : b[t];
+        ss = fmaf(u[t], u[t], ss);
+      }
+      store8(B, i, 1, b);
+      store8(a.X, xoff + i, a.x_f32, u);
+    }
+  } else {
+    for (long long i = static_cast<long long>(blockIdx.x) * EW_THREADS + threadIdx.x; i < numel;
+         i += static_cast<long long>(gridDim.x) * EW_THREADS) {
+      const long long r = i / a.cols, c = i % a.cols;
+      const float g = load_elem(G, i, a.g_f32);
+      const float b = fmaf(mu, B[i], g);
+      const float u = a.nesterov ? fmaf(mu, b, g) : b;
+      B[i] = b;
+      ss = fmaf(u, u, ss);
+      store_elem(a.X, xoff + r * a.ldx + c, u, a.x_f32);
+    }
+  }
+  const float tot = block_sum(ss, red);
+  if (threadIdx.x == 0) a.partials[static_cast<long long>(l) * a.nblk + blockIdx.x] = tot;
+}
+
+// Tall (rows > cols) matrices: X = U^T (cols x rows), through a 64x64 tile.
+constexpr int TT = 64;
+__global__ void __launch_bounds__(EW_THREADS) momentum_tall_kernel(const MomentumArgs a) {
+  __shared__ float tile[TT][TT + 1];
+  __shared__ float red[EW_THREADS / 32];
+  const int l = blockIdx.y;
+  const void* G = a.G[l];
+  float* B = static_cast<float*>(a.B[l]);
+  const long long xoff = static_cast<long long>(l) * a.cols * a.ldx;  // X is cols x rows, row stride ldx
+  const int tr = (a.rows + TT - 1) / TT, tc = (a.cols + TT - 1) / TT;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
+  const float mu = a.mu;
+  float ss = 0.f;
+  for (int t = blockIdx.x; t < tr * tc; t += gridDim.x) {
+    const int r0 = (t / tc) * TT, c0 = (t % tc) * TT;
+    // read rows r0..r0+63 of the stored matrix, two columns per thread
+#pragma unroll
+    for (int k = 0; k < TT / 8; ++k) {
+      const int rr = ty + 8 * k;
+      const int r = r0 + rr;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int cc = 2 * tx + h;
+        const int c = c0 + cc;
+        float u = 0.f;
+        if (r < a.rows && c < a.cols) {
+          const long long i = static_cast<long long>(r) * a.cols + c;
+          const float g = load_elem(G, i, a.g_f32);
+          const float b = fmaf(mu, B[i], g);
+          u = a.nesterov ? fmaf(mu, b, g) : b;
+          B[i] = b;
+          ss = fmaf(u, u, ss);
+        }
+        tile[rr][cc] = u;
+      }
+    }
+    __syncthreads();
+    // write X rows c0..c0+63 (= stored columns), columns r0..r0+63
+#pragma unroll
+    for (int k = 0; k < TT / 8; ++k) {
+      const int cc = ty + 8 * k;
+      const int xr = c0 + cc;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int rr = 2 * tx + h;
+        const int xc = r0 + rr;
+        if (xr < a.cols && xc < a.rows) store_elem(a.X, xoff + static_cast<long long>(xr) * a.ldx + xc, tile[rr][cc], a.x_f32);
+      }
+    }
+    __syncthreads();
+  }
+  const float tot = block_sum(ss, red);
+  if (threadIdx.x == 0) a.partials[static_cast<long long>(l) * a.nblk + blockIdx.x] = tot;
+}
+
+__global__ void norm_finalize_kernel(const float* __restrict__ partials, int nblk, float eps, float* s, float* s2) {
+  const int l = blockIdx.x;
+  __shared__ double red[32];
+  double acc = 0.0;
+  for (int i = threadIdx.x; i < nblk; i += blockDim.x) acc += static_cast<double>(partials[static_cast<long long>(l) * nblk + i]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t += red[w];
+    const double inv = 1.0 / (sqrt(t) + static_cast<double>(eps));
+    s[l] = static_cast<float>(inv);
+    s2[l] = static_cast<float>(inv * inv);
+  }
+}
+
+__global__ void __launch_bounds__(256) scale_epilogue_kernel(const void* X, long long ldx, int x_f32, int m, int n,
+                                                             const float* s, const Epilogue epi) {
+  const int l = blockIdx.z;
+  const int row = blockIdx.y * 8 + (threadIdx.x >> 5);
+  const int col = blockIdx.x * 32 + (threadIdx.x & 31);
+  if (row >= m) return;
+  float v[1];
+  v[0] = (col < n) ? s[l] * load_elem(X, static_cast<long long>(l) * m * ldx + static_cast<long long>(row) * ldx + col, x_f32) : 0.f;
+  if (col < n) epilogue_row<1>(epi, l, row, col, v, m, n);
+}
+
+__global__ void diff_norms_kernel(const void* X, const void* Y, long long ld, int m, int n, int is_f32,
+                                  double* acc) {
+  const int l = blockIdx.y;
+  double d = 0.0, y2 = 0.0;
+  const long long numel = static_cast<long long>(m) * n;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < numel;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long r = i / n, c = i % n;
+    const long long o = static_cast<long long>(l) * m * ld + r * ld + c;
+    const double x = load_elem(X, o, is_f32), y = load_elem(Y, o, is_f32);
+    d += (x - y) * (x - y);
+    y2 += y * y;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    d += __shfl_xor_sync(0xffffffffu, d, o);
+    y2 += __shfl_xor_sync(0xffffffffu, y2, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    atomicAdd(&acc[0], d);
+    atomicAdd(&acc[1], y2);
+  }
+}
+
+}  // namespace
+
+int momentum_partials(int rows, int cols, int cnt, int num_sms) {
+  const long long numel = static_cast<long long>(rows) * cols;
+  long long want = (4LL * num_sms + cnt - 1) / cnt;  // ~4 blocks per SM over the group
+  long long cap;
+  if (rows > cols)
+    cap = static_cast<long long>((rows + TT - 1) / TT) * ((cols + TT - 1) / TT);
+  else
+    cap = (numel + EW_THREADS * VEC * 4 - 1) / (EW_THREADS * VEC * 4);  // >= 4 vectors per thread
+  long long nb = want < cap ? want : cap;
+  if (nb < 1) nb = 1;
+  if (nb > 4096) nb = 4096;
+  return static_cast<int>(nb);
+}
+
+cudaError_t launch_momentum(const MomentumArgs& a, cudaStream_t s) {
+  if (a.cnt <= 0) return cudaSuccess;
+  if (a.cnt > 65535) return cudaErrorInvalidValue;
+  dim3 grid(a.nblk, a.cnt);
+  if (a.transposed) {
+    momentum_tall_kernel<<<grid, EW_THREADS, 0, s>>>(a);
+  } else {
+    // The vector path needs cols % 8 == 0 (then ldx == cols) and 16-byte
+    // aligned G/B bases (checked by the host: a.aligned).
+    const int vec_ok = (a.cols % VEC == 0) && (a.ldx == a.cols) && a.aligned ? 1 : 0;
+    momentum_wide_kernel<<<grid, EW_THREADS, 0, s>>>(a, vec_ok);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_norm_finalize(const float* partials, int nblk, int cnt, float eps, float* s, float* s2,
+                                 cudaStream_t st) {
+  if (cnt <= 0) return cudaSuccess;
+  norm_finalize_kernel<<<cnt, 256, 0, st>>>(partials, nblk, eps, s, s2);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scale_epilogue(const void* X, long long ldx, int x_f32, int m, int n, int cnt, const float* s,
+                                  const Epilogue& epi, cudaStream_t st) {
+  if (cnt <= 0) return cudaSuccess;
+  if (cnt > 65535 || (m + 7) / 8 > 65535) return cudaErrorInvalidValue;
+  dim3 grid((n + 31) / 32, (m + 7) / 8, cnt);
+  scale_epilogue_kernel<<<grid, 256, 0, st>>>(X, ldx, x_f32, m, n, s, epi);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_diff_norms(const void* X, const void* Y, long long ld, int m, int n, int cnt, int is_f32,
+                              double* acc, cudaStream_t st) {
+  if (cnt <= 0) return cudaSuccess;
+  dim3 grid(64, cnt);
+  diff_norms_kernel<<<grid, 256, 0, st>>>(X, Y, ld, m, n, is_f32, acc);
+  return cudaGetLastError();
+}
+
+}  // namespace dmuon

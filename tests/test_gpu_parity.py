@@ -1,0 +1,143 @@
+"""CUDA path against the fp64 oracle on seeded inputs (through the C ABI).
+
+Bars: the update O within 3e-2 relative Frobenius error on the bf16
+tensor-core path and 1e-4 on the fp32 path, per matrix; the momentum buffer
+within 1e-6 relative, elementwise; the parameter write equal to the oracle's
+apply of the GPU's own update within one rounding of the parameter dtype.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.muon_oracle as ora
+from parity_helpers import (check_momentum, gpu_step, gpu_update, make_inputs, oracle_update, rel_fro, to64)
+
+pytestmark = pytest.mark.gpu
+
+BF16_TOL = 3e-2
+F32_TOL = 1e-4
+
+SMALL_SHAPES = [
+    [(64, 256)] * 3,            # tiny wide, several per group
+    [(96, 200)] * 2,            # ragged: no dimension a tile multiple
+    [(300, 130)] * 2,           # tall and ragged: transposed iterate
+    [(128, 128)],               # square
+    [(256, 1024), (64, 256), (1024, 256)],  # mixed groups in one call
+    [(200, 520), (520, 200)],   # a wide/tall pair
+    [(17, 33)],                 # odd sizes (strides padded in scratch)
+    [(1, 64), (64, 1)],         # single row / column
+]
+
+
+def _wide_enough(shapes):
+    """The Gram-space form squares the condition number; in bf16 it holds the
+    bar only for clearly rectangular matrices (the autotuner offers it from
+    n >= 1.25 m and gates it on accuracy)."""
+    return all(max(r, c) >= 1.9 * min(r, c) for r, c in shapes)
+
+
+CASES = [(s, v) for s in SMALL_SHAPES for v in ("direct", "gram", "auto")
+         if v != "gram" or _wide_enough(s)]
+
+
+@pytest.mark.parametrize("shapes,variant", CASES,
+                         ids=["+".join(f"{r}x{c}" for r, c in s) + "-" + v for s, v in CASES])
+def test_bf16_update_matches_oracle(dmuon_lib, shapes, variant):
+    Ws, Gs, Ms = make_inputs(shapes, seed=11, m_std=1e-3)
+    Os, Bn = gpu_update(dmuon_lib, Gs, Ms, variant=variant)
+    for i in range(len(shapes)):
+        Bo, Oo = oracle_update(Gs[i], Ms[i])
+        e = rel_fro(to64(Os[i]), Oo)
+        assert e <= BF16_TOL, (shapes[i], variant, e)
+        check_momentum(Bn[i], Gs[i], Ms[i], 0.95)
+
+
+def test_fp32_single_256x512_matches_oracle(dmuon_lib):
+    """The fp32 workload: one 256x512 fp32 weight, W, G, M ~ N(0, 0.02^2), seed 0."""
+    from newton_schulz_normalise_b200 import workloads as wl
+    w = wl.WORKLOADS["single-256x512-fp32"]
+    Ws, Gs, Ms = wl.generate(w, device="cuda")
+    Os, Bn = gpu_update(dmuon_lib, Gs, Ms, mu=w.mu, steps=w.ns_steps)
+    Bo, Oo = oracle_update(Gs[0], Ms[0], w.mu, w.ns_steps)
+    e = rel_fro(to64(Os[0]), Oo)
+    assert e <= F32_TOL, e
+    check_momentum(Bn[0], Gs[0], Ms[0], w.mu)
+    Wg, Mg = gpu_step(dmuon_lib, Ws, Gs, Ms, w.lr, w.wd, w.mu, w.ns_steps)
+    Wo, _, _ = ora.muon_step(to64(Ws[0]), to64(Gs[0]), to64(Ms[0]), w.lr, w.wd, w.mu, w.ns_steps)
+    # fp32 parameters: the write differs from the oracle by lr*scale*|dO| + fp32 rounding
+    scale = w.lr * ora.rms_scale(256, 512)
+    dW = np.abs(to64(Wg[0]) - Wo)
+    assert dW.max() <= scale * np.abs(to64(Os[0]) - Oo).max() * 1.01 + 2 ** -23 * np.abs(Wo).max() * 2
+
+
+@pytest.mark.parametrize("steps", [0, 1, 2, 5, 7])
+def test_ns_steps(dmuon_lib, steps):
+    shapes = [(96, 200), (200, 96)]
+    Ws, Gs, Ms = make_inputs(shapes, seed=23)
+    for variant in ("direct", "gram"):
+        Os, _ = gpu_update(dmuon_lib, Gs, Ms, steps=steps, variant=variant)
+        for i in range(2):
+            _, Oo = oracle_update(Gs[i], Ms[i], steps=steps)
+            assert rel_fro(to64(Os[i]), Oo) <= BF16_TOL, (steps, variant, i)
+
+
+def test_plain_momentum_and_custom_eps(dmuon_lib):
+    shapes = [(128, 384)]
+    Ws, Gs, Ms = make_inputs(shapes, seed=5, m_std=2e-3)
+    Os, Bn = gpu_update(dmuon_lib, Gs, Ms, mu=0.9, nesterov=False, eps=1e-3)
+    Bo, Oo = ora.muon_update(to64(Gs[0]), to64(Ms[0]), 0.9, 5, 1e-3, False)
+    assert rel_fro(to64(Os[0]), Oo) <= BF16_TOL
+    check_momentum(Bn[0], Gs[0], Ms[0], 0.9)
+
+
+def test_zero_gradient_leaves_decay_only(dmuon_lib):
+    W = (torch.randn(64, 256, device="cuda") * 0.02).bfloat16()
+    G = torch.zeros(64, 256, device="cuda", dtype=torch.bfloat16)
+    M = torch.zeros(64, 256, device="cuda", dtype=torch.float32)
+    Wg, Mg = gpu_step(dmuon_lib, [W], [G], [M], lr=0.02, wd=0.1, mu=0.95)
+    expect = to64(W) * (1 - 0.02 * 0.1)
+    assert np.all(np.abs(to64(Wg[0]) - expect) <= np.abs(expect) * 2.0 ** -8)
+    assert torch.count_nonzero(Mg[0]) == 0
+
+
+@pytest.mark.parametrize("shapes", [[(64, 256)] * 2, [(300, 130)], [(1024, 1024)]],
+                         ids=["64x256x2", "300x130", "1024sq"])
+def test_bf16_step_write_matches_oracle_apply(dmuon_lib, shapes):
+    """The fused parameter write equals the oracle's apply of the GPU update,
+    within one bf16 rounding; and W' is within the update tolerance of the
+    oracle's full step."""
+    lr, wd, mu = 0.02, 0.1, 0.95
+    Ws, Gs, Ms = make_inputs(shapes, seed=31, m_std=1e-3)
+    Os, _ = gpu_update(dmuon_lib, Gs, Ms, mu=mu)
+    Wg, _ = gpu_step(dmuon_lib, Ws, Gs, Ms, lr, wd, mu)
+    for i, (r, c) in enumerate(shapes):
+        w_apply = ora.apply_update(to64(Ws[i]), to64(Os[i]), lr, wd)
+        # one bf16 rounding of the result plus fp32 evaluation error of the
+        # two terms (which can cancel)
+        terms = np.abs((1 - lr * wd) * to64(Ws[i])) + np.abs(lr * ora.rms_scale(r, c) * to64(Os[i]))
+        bound = np.abs(w_apply) * 2.0 ** -8 + terms * 1e-6
+        assert np.all(np.abs(to64(Wg[i]) - w_apply) <= bound), i
+        Wo, _, Oo = ora.muon_step(to64(Ws[i]), to64(Gs[i]), to64(Ms[i]), lr, wd, mu)
+        scale = lr * ora.rms_scale(r, c)
+        bound = scale * BF16_TOL * np.linalg.norm(Oo) + 2.0 ** -8 * np.linalg.norm(Wo)
+        assert np.linalg.norm(to64(Wg[i]) - Wo) <= bound
+
+
+def test_deterministic(dmuon_lib):
+    shapes = [(256, 1024)] * 4
+    Ws, Gs, Ms = make_inputs(shapes, seed=41)
+    a, _ = gpu_step(dmuon_lib, Ws, Gs, Ms)
+    b, _ = gpu_step(dmuon_lib, Ws, Gs, Ms)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_gram_and_direct_agree_on_wide(dmuon_lib):
+    shapes = [(256, 1024)] * 2
+    _, Gs, Ms = make_inputs(shapes, seed=43)
+    Od, _ = gpu_update(dmuon_lib, Gs, Ms, variant="direct")
+    Og, _ = gpu_update(dmuon_lib, Gs, Ms, variant="gram")
+    for i in range(2):
+        assert rel_fro(to64(Og[i]), to64(Od[i])) <= 2e-2
