@@ -1,0 +1,387 @@
+#!/usr/bin/env python
+"""Benchmark of the Muon / DMuon optimizer step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one call of the library's ``dmuon_step`` over a whole parameter set
+(momentum, normalisation, 5 quintic Newton-Schulz steps, scale, decay and the
+parameter write for every matrix).  Default workload: 64 square 1024 x 1024
+bf16 weights with fp32 momenta (grads ~ N(0, 1e-3^2)).  Inputs are resident
+in HBM before the timed region; they total 537 MB (> 126 MB of L2), so no L2
+flush is needed between steps.
+
+Prints one JSON line (rank 0).  N > 1 runs independent replicas, one per
+rank (the step has no exchange on one parameter set); timing is the max over
+ranks of the device-timed region.  ``--impl reference`` times the fp64 CPU
+oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "Muon step ms per param set; NS TFLOPS as % of B200 bf16 dense peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def measured_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        d["_source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["_source"] = "fallback"
+    return d
+
+
+def ns_flops(rows, cols, steps, variant):
+    m, n = min(rows, cols), max(rows, cols)
+    if steps == 0:
+        return 0.0
+    if variant == "gram":
+        return 2.0 * (2 * m * m * n + (1 + 4 * (steps - 1)) * m ** 3)
+    return 2.0 * steps * (2 * m * m * n + m ** 3)
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampled every 100 ms in a background process; samples are
+    kept with host timestamps so only those inside the timed window count."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = [s for t, s in self.samples if t0 <= t <= t1]
+        if not rows:  # a short window: take the nearest samples around it
+            rows = [s for t, s in self.samples if t0 - 0.3 <= t <= t1 + 0.3]
+        mhz, maxmhz, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            f = [x.strip() for x in r.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                maxmhz = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": maxmhz, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ------------------------------------------------------------------ CPU baseline (oracle)
+def cpu_baseline(w, budget_s=12.0):
+    """The fp64 oracle as it stands, on the first matrices of the workload,
+    as many as fit in ~budget_s, extrapolated to the whole parameter set."""
+    import numpy as np
+    import torch
+    import oracle.muon_oracle as ora
+    from newton_schulz_normalise_b200 import workloads as wl
+
+    shapes = w.shapes()
+    cores = len(os.sched_getaffinity(0))
+    torch.set_num_threads(cores)
+    done, spent = 0, 0.0
+    per_shape = {}
+    for i, (r, c) in enumerate(shapes):
+        if (r, c) in per_shape and len(per_shape[(r, c)]) >= 2:
+            continue
+        Ws, Gs, Ms = wl.generate(w, device="cpu", indices=[i])
+        W = Ws[0].double().numpy()
+        G = Gs[0].double().numpy()
+        M = Ms[0].double().numpy()
+        t0 = time.perf_counter()
+        ora.muon_step(W, G, M, w.lr, w.wd, w.mu, w.ns_steps)
+        dt = time.perf_counter() - t0
+        per_shape.setdefault((r, c), []).append(dt)
+        done += 1
+        spent += dt
+        if spent > budget_s:
+            break
+    total_s = 0.0
+    for (r, c) in shapes:
+        ts = per_shape.get((r, c))
+        if ts is None:  # not reached within budget: scale by flops from a timed shape
+            (r0, c0), t0s = next(iter(per_shape.items()))
+            ts = [statistics.mean(t0s) * ns_flops(r, c, 5, "direct") / ns_flops(r0, c0, 5, "direct")]
+        total_s += statistics.mean(ts)
+    return {
+        "value": total_s * 1e3, "unit": "ms", "cores": cores, "kind": "oracle",
+        "sample": f"{done} of {len(shapes)} matrices timed one by one (fp64 numpy, BLAS on "
+                  f"{cores} threads), mean per shape x count",
+        "cpu": _cpu_model(),
+    }
+
+
+def _cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# ------------------------------------------------------------------ distributed
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def run_reference(args, w):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    times = []
+    base = None
+    for _ in range(args.warmup + args.steps):
+        # each step times at least one matrix; the whole run stays near 2 minutes
+        base = cpu_baseline(w, budget_s=max(0.3, 120.0 / max(args.steps + args.warmup, 1)))
+        times.append(base["value"])
+    val = statistics.mean(times[args.warmup:]) if len(times) > args.warmup else times[-1]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "ms", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": val, "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "matrices": len(w.shapes())},
+        "cpu_baseline": {"value": val, "unit": "ms", "cores": base["cores"], "kind": "oracle",
+                         "sample": base["sample"]},
+        "e2e": {"value": val, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def profile_traffic(kernel_file: Path):
+    """Per-launch DRAM traffic of the dominant kernel from the committed ncu
+    summary, if it was taken on the current kernel source."""
+    import hashlib
+    summ = ROOT / "profiles" / "tc_gemm_batch64-1024x1024.md"
+    if not summ.exists():
+        return None
+    sha = hashlib.sha256(kernel_file.read_bytes()).hexdigest()[:16]
+    txt = summ.read_text()
+    src, traffic = None, None
+    for line in txt.splitlines():
+        if line.startswith("kernel_source_sha256_16:"):
+            src = line.split(":", 1)[1].strip()
+        if line.startswith("traffic_bytes_per_launch:"):
+            traffic = float(line.split(":", 1)[1].strip())
+    return traffic if src == sha else None
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="batch64-1024x1024-bf16")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    from newton_schulz_normalise_b200 import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+    from newton_schulz_normalise_b200 import binding as B
+
+    ws, rank, local = dist_env()
+    if ws != args.gpus and rank == 0:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={ws}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", init_method="env://", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+
+    Ws, Gs, Ms = wl.generate(w, device=dev)
+    shapes = w.shapes()
+    pdt = B.DMUON_BF16 if w.param_dtype == "bf16" else B.DMUON_F32
+    opts = B.options(pdt, pdt)
+
+    def step():
+        B.dmuon_step_ex(Ws, Gs, Ms, w.lr, w.wd, w.mu, w.ns_steps, opts=opts, stream=stream)
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+
+    # warm-up (first call tunes each shape group and fills the cache)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    plans = B.dmuon_cache_entries()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    # ---------------- device-timed region: K steps
+    barrier()
+    torch.cuda.synchronize()
+    l0 = B.dmuon_launch_count()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_host0 = time.time()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    t_host1 = time.time()
+    barrier()
+    launches = (B.dmuon_launch_count() - l0) // args.steps
+    ms = ev0.elapsed_time(ev1)
+    time.sleep(0.2)
+    clocks.stop()
+    clk = clocks.summary(t_host0, t_host1)
+
+    # ---------------- per-kernel timing pass (same steps, events around each launch)
+    B.dmuon_timing_reset()
+    B.dmuon_timing_enable(True)
+    kt_steps = min(args.steps, 50)
+    for _ in range(kt_steps):
+        step()
+    torch.cuda.synchronize()
+    B.dmuon_timing_enable(False)
+    kinds = {k: B.dmuon_timing_get(k) for k in (B.KIND_TC_GEMM, B.KIND_EW, B.KIND_SIMT_GEMM, B.KIND_OTHER)}
+    B.dmuon_timing_reset()
+
+    # ---------------- end to end through the C ABI with host buffers
+    # Each step: grads H2D from pinned host memory, the step, params D2H.
+    hG = [g.cpu().pin_memory() for g in Gs]
+    hW = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in Ws]
+    h2d = sum(x.numel() * x.element_size() for x in hG)
+    d2h = sum(x.numel() * x.element_size() for x in hW)
+    e2e_steps = max(3, min(args.steps, 20))
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for d, h in zip(Gs, hG):
+            d.copy_(h, non_blocking=True)
+        step()
+        for h, d in zip(hW, Ws):
+            h.copy_(d, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    # ---------------- reduce over ranks (max), report on rank 0
+    vals = torch.tensor([ms, e2e_ms], device=dev, dtype=torch.float64)
+    if ws > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    ms_max, e2e_max = vals.tolist()
+    ms_per_step = ms_max / args.steps
+    value = ms_per_step / ws  # N replicas each process one parameter set per step
+
+    peaks = measured_peaks()
+    variants = {}
+    for e in plans:  # "rows cols dtype steps variant bn cnt cost"
+        f = e.split()
+        variants[(int(f[0]), int(f[1]))] = f[4]
+    flops = sum(ns_flops(r, c, w.ns_steps, variants.get((r, c), "direct")) for r, c in shapes)
+    tflops = flops / (ms_per_step * 1e-3) / 1e12
+    gemm = kinds[B.KIND_TC_GEMM]
+    peak_tc = peaks["bf16_tflops"]
+    ach = gemm["flops"] / (gemm["ms"] * 1e-3) / 1e12 if gemm["ms"] > 0 else 0.0
+    traffic = profile_traffic(ROOT / "newton_schulz_normalise_b200" / "csrc" / "gemm_tc.cu")
+    ew = kinds[B.KIND_EW]
+    ew_gbs = ew["bytes"] / (ew["ms"] * 1e-3) / 1e9 if ew["ms"] > 0 else 0.0
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 4), "unit": "ms", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,0.02^2) weights, N(0,1e-3^2) grads, zero fp32 momenta)",
+            "config": {"workload": w.name, "matrices": len(shapes),
+                       "shapes": sorted({f"{r}x{c}" for r, c in shapes}), "ns_steps": w.ns_steps,
+                       "lr": w.lr, "wd": w.wd, "mu": w.mu, "parallelism": f"replicas{ws}",
+                       "l2": "inputs 537 MB > 126 MB L2, no flush between steps",
+                       "plans": plans},
+            "ns_tflops": round(tflops, 1),
+            "ns_frac_of_peak": round(tflops / peak_tc, 4),
+            "roofline": {"bound": "tensor", "kernel": "tc_gemm_kernel", "achieved": round(ach, 1),
+                         "peak": peak_tc, "unit": "TFLOP/s", "frac": round(ach / peak_tc, 4),
+                         "traffic": traffic, "peak_source": f"{peaks['_source']} bf16_tflops (burst)",
+                         "launches": gemm["launches"] // kt_steps,
+                         "share_of_step": round(gemm["ms"] / kt_steps / ms_per_step, 3) if ms_per_step else None},
+            "elementwise": {"bound": "hbm", "kernel": "momentum", "achieved": round(ew_gbs, 1),
+                            "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": round(ew_gbs / peaks["hbm_gbs"], 4)},
+            "e2e": {"value": round(e2e_max / ws, 4), "unit": "ms", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches * args.steps,
+            "gpu_launches_per_step": launches,
+            "clocks": clk,
+        }
+        if not args.no_cpu_baseline and ws == 1:
+            line["cpu_baseline"] = cpu_baseline(w)
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
