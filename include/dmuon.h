@@ -124,6 +124,32 @@ int dmuon_compute_update(const void* const* grads, void* const* momenta,
                          const dmuon_options* opts, float* const* out, void* stream);
 
 /*
+ * dmuon_compute_update_noalloc -- dmuon_compute_update for ONE matrix that
+ * allocates nothing.  No counterpart on the pages: it exists for callers that
+ * cannot allocate device memory inside their step, e.g. a framework whose
+ * caching allocator owns all of device memory and forbids outside cudaMalloc,
+ * or a loop that cannot take the device-wide synchronisation that
+ * cudaMalloc/cudaFree imply.  (dmuon_set_workspace is the other route.)
+ *   grad      device, rows x cols row-major (dtype opts->grad_dtype); read only.
+ *   momentum  device, rows x cols fp32; updated in place (B').
+ *   out       device, rows x cols fp32: the update O, as dmuon_compute_update.
+ * Scratch is a fixed 64 MiB array in the library's device image, held by
+ * every GPU that loads the library until the process exits.  A matrix whose
+ * scratch exceeds it (about 4M bf16 elements for a square matrix, more for
+ * wide ones) is rejected with DMUON_ERR_INVALID before any launch.  The
+ * first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  It uses the plan the autotuner cached for this shape (count 1)
+ * when there is one, else the direct form; it never autotunes.  All calls
+ * share the one array and it keeps the last call's contents (each call
+ * clears the words it reads before writing them): calls whose GPU work
+ * overlaps, e.g. on two streams without ordering between them, race.
+ * Calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows, int64_t cols, float mu,
+                                 int ns_steps, const dmuon_options* opts, float* out, void* stream);
+
+/*
  * dmuon_gemm_bf16 -- the tensor-core GEMM core on its own (tests, tuning):
  *   D[l] = alpha * A[l] * op(B[l]) + beta * C[l]            l = 0..batch-1
  * A: device bf16, M x K row-major (K contiguous), leading dim lda, batch

@@ -32,7 +32,7 @@ EXPORTS = (
     "dmuon_gemm_bf16", "dmuon_cache_save", "dmuon_cache_load", "dmuon_cache_clear",
     "dmuon_cache_size", "dmuon_cache_entry", "dmuon_set_workspace", "dmuon_workspace_size",
     "dmuon_timing_enable", "dmuon_timing_reset", "dmuon_timing_get", "dmuon_launch_count",
-    "dmuon_last_error", "dmuon_version",
+    "dmuon_last_error", "dmuon_version", "dmuon_compute_update_noalloc",
 )
 
 
@@ -77,6 +77,7 @@ def _load() -> ctypes.CDLL:
         "dmuon_launch_count": (I64, []),
         "dmuon_last_error": (ctypes.c_char_p, []),
         "dmuon_version": (I, []),
+        "dmuon_compute_update_noalloc": (I, [P, P, I64, I64, F, I, ctypes.POINTER(Options), P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -176,6 +177,21 @@ def dmuon_compute_update(grads, momenta, out, mu, ns_steps=5, opts: Options | No
         opts = options(dt, dt, **kw)
     return _check(lib.dmuon_compute_update(_ptrs(grads), _ptrs(momenta), _shapes(grads), n, mu, ns_steps,
                                            ctypes.byref(opts), _ptrs(out), _stream(stream)))
+
+
+def dmuon_compute_update_noalloc(grad, momentum, out, mu, ns_steps=5, opts: Options | None = None,
+                                 stream=None, **kw):
+    """dmuon_compute_update for one matrix with the library's static scratch
+    (no device allocation)."""
+    if grad.dim() != 2 or not grad.is_contiguous():
+        raise ValueError("expected a contiguous 2-D gradient")
+    if opts is None:
+        dt = _dtype_code(grad)
+        opts = options(dt, dt, **kw)
+    rows, cols = grad.shape
+    return _check(lib.dmuon_compute_update_noalloc(grad.data_ptr(), momentum.data_ptr(), rows, cols, mu,
+                                                   ns_steps, ctypes.byref(opts), out.data_ptr(),
+                                                   _stream(stream)))
 
 
 def dmuon_gemm_bf16(A, B, D, alpha=1.0, beta=0.0, C=None, b_kmajor=True, bn=0, stream=None):

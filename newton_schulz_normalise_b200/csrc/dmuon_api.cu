@@ -822,6 +822,42 @@ Hyper hyper_from(float lr, float wd, float mu, int steps, const dmuon_options& o
 }
 
 }  // namespace
+
+// ------------------------------------------------------------------ no-alloc entry point
+// Scratch of dmuon_compute_update_noalloc: a fixed array in the library's own
+// device image, so that entry point never allocates.  Every GPU that loads
+// the library holds these 64 MiB until the process exits.  Host code must not
+// use the symbol's name as an address; it asks the runtime for the device
+// address once per device (static_scratch below).
+constexpr size_t kStaticScratchBytes = size_t(64) << 20;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_addr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device; looked up with
+// cudaGetSymbolAddress on the first call per device (with that device current).
+int static_scratch(void** out, int* device) {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(DMUON_ERR_INVALID, "device ordinal %d not supported", dev);
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  if (!g_static_addr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(DMUON_ERR_CUDA, "cudaGetSymbolAddress(static scratch) on device %d: %s", dev, cudaGetErrorString(e));
+    g_static_addr[dev] = p;
+  }
+  *out = g_static_addr[dev];
+  *device = dev;
+  return DMUON_OK;
+}
+
+}  // namespace
 }  // namespace dmuon
 
 using namespace dmuon;
@@ -868,6 +904,77 @@ int dmuon_compute_update(const void* const* grads, void* const* momenta, const i
   Request r{nullptr, grads, momenta, out, shapes, count, hyper_from(0.f, 0.f, mu, ns_steps, o), o,
             static_cast<cudaStream_t>(stream)};
   return run_step(r);
+}
+
+int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows, int64_t cols, float mu,
+                                 int ns_steps, const dmuon_options* opts, float* out, void* stream) {
+  t_err.clear();
+  dmuon_options o;
+  dmuon_options_init(&o);
+  if (opts) o = *opts;
+  if (!grad || !momentum || !out) return fail(DMUON_ERR_INVALID, "null pointer");
+  const int64_t shape[2] = {rows, cols};
+  void* gp = const_cast<void*>(grad);
+  float* op = out;
+  Request r{nullptr, reinterpret_cast<const void* const*>(&gp), &momentum, &op, shape, 1,
+            hyper_from(0.f, 0.f, mu, ns_steps, o), o, static_cast<cudaStream_t>(stream)};
+  int rc = validate(r);
+  if (rc) return rc;
+  const bool f32 = o.param_dtype == DMUON_F32;
+  // plan: the one the autotuner cached for this shape, else the direct form
+  Plan plan;
+  if (o.variant == DMUON_VARIANT_DIRECT || o.variant == DMUON_VARIANT_GRAM) plan.variant = o.variant;
+  {
+    std::lock_guard<std::mutex> lk(g_cache_mu);
+    auto it = g_cache.find(Key{rows, cols, f32 ? 1 : 0, ns_steps, 1});
+    if (it != g_cache.end() && (o.variant == DMUON_VARIANT_AUTO || it->second.variant == o.variant)) plan = it->second;
+  }
+  void* base = nullptr;
+  int dev = 0;
+  rc = static_scratch(&base, &dev);
+  if (rc) return rc;
+  int sms = 0;
+  CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  const Geo g = make_geo(rows, cols, f32);
+  const int nblk = momentum_partials(g.rows, g.cols, 1, sms);
+  const Layout L = make_layout(g, 1, nblk);
+  const size_t header = 256;  // 4 pointer slots and the device error word
+  const size_t need = header + L.total;
+  if (need > kStaticScratchBytes)
+    return fail(DMUON_ERR_INVALID,
+                "a %lld x %lld %s matrix needs %zu bytes of scratch; dmuon_compute_update_noalloc has %zu",
+                (long long)rows, (long long)cols, f32 ? "fp32" : "bf16", need, kStaticScratchBytes);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* sb = static_cast<uint8_t*>(base);
+  void* tables[4] = {gp, momentum, nullptr, out};
+  CUDA_TRY(cudaMemcpyAsync(sb, tables, sizeof(tables), cudaMemcpyHostToDevice, s));
+  int* dev_err = reinterpret_cast<int*>(sb + 64);
+  CUDA_TRY(cudaMemsetAsync(dev_err, 0, sizeof(int), s));  // the only word read before it is written
+  DeviceCtx c;  // launch parameters only: nothing is allocated for it
+  c.device = dev;
+  c.num_sms = sms;
+  c.err_dev = dev_err;
+  Chunk ch;
+  ch.g = &g;
+  ch.cnt = 1;
+  ch.base = sb + header;
+  ch.L = L;
+  void** dtab = reinterpret_cast<void**>(sb);
+  ch.Gt = dtab;
+  ch.Bt = dtab + 1;
+  ch.Wt = dtab + 2;
+  ch.Ot = reinterpret_cast<float* const*>(dtab + 3);
+  ch.nblk = nblk;
+  ch.aligned = aligned16(grad) && aligned16(momentum);
+  rc = run_momentum(c, ch, f32, o.grad_dtype == DMUON_F32, r.h, s);
+  if (rc) return rc;
+  Epilogue fin{};
+  fin.mode = EPI_OUT;
+  fin.Out = ch.Ot;
+  fin.transposed = g.transposed;
+  fin.ldw = g.cols;
+  fin.w_f32 = f32;
+  return run_ns(c, ch, f32, plan.variant, plan.bn, r.h, fin, 1, s);
 }
 
 int dmuon_gemm_bf16(const void* A, int64_t lda, int64_t sa, const void* B, int64_t ldb, int64_t sb, int b_kmajor,
