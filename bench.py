@@ -338,9 +338,12 @@ def main():
     for e in plans:  # "rows cols dtype steps variant bn cnt cost"
         f = e.split()
         variants[(int(f[0]), int(f[1]))] = f[4]
-    flops = sum(ns_flops(r, c, w.ns_steps, variants.get((r, c), "direct")) for r, c in shapes)
-    tflops = flops / (ms_per_step * 1e-3) / 1e12
     gemm = kinds[B.KIND_TC_GEMM]
+    simt = kinds[B.KIND_SIMT_GEMM]
+    # executed NS FLOPs per step (symmetric products count their computed tiles only)
+    flops = (gemm["flops"] + simt["flops"]) / kt_steps
+    dense = sum(ns_flops(r, c, w.ns_steps, variants.get((r, c), "direct")) for r, c in shapes)
+    tflops = flops / (ms_per_step * 1e-3) / 1e12
     peak_tc = peaks["bf16_tflops"]
     ach = gemm["flops"] / (gemm["ms"] * 1e-3) / 1e12 if gemm["ms"] > 0 else 0.0
     traffic = profile_traffic(ROOT / "newton_schulz_normalise_b200" / "csrc" / "gemm_tc.cu")
@@ -360,6 +363,7 @@ def main():
                        "plans": plans},
             "ns_tflops": round(tflops, 1),
             "ns_frac_of_peak": round(tflops / peak_tc, 4),
+            "ns_tflops_dense_equivalent": round(dense / (ms_per_step * 1e-3) / 1e12, 1),
             "roofline": {"bound": "tensor", "kernel": "tc_gemm_kernel", "achieved": round(ach, 1),
                          "peak": peak_tc, "unit": "TFLOP/s", "frac": round(ach / peak_tc, 4),
                          "traffic": traffic, "peak_source": f"{peaks['_source']} bf16_tflops (burst)",

@@ -157,12 +157,16 @@ int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows,
  *    (op(B) = B^T), b_kmajor = 0: stored K x N (op(B) = B).  C, D: device
  *    bf16 M x N (C may be NULL => beta ignored).  All leading dims and batch
  *    strides must be multiples of 8 elements and pointers 16-byte aligned.
- *    bn selects the tile width (128 or 256; 0 = default).
+ *    tile: 128 or 256 = one CTA per 128 x tile output tile, 512 = a CTA pair
+ *    (tcgen05 cta_group::2) per 256 x 256 tile, 0 = 256.
+ *    sym = 1 (needs M == N) declares the result symmetric: only the tiles
+ *    that meet the upper triangle are computed and each element (r, c >= r)
+ *    is also written to (c, r).
  */
 int dmuon_gemm_bf16(const void* A, int64_t lda, int64_t sa, const void* B, int64_t ldb,
                     int64_t sb, int b_kmajor, const void* C, int64_t ldc, int64_t sc,
                     void* D, int64_t ldd, int64_t sd, int M, int N, int K, int batch,
-                    float alpha, float beta, int bn, void* stream);
+                    float alpha, float beta, int tile, int sym, void* stream);
 
 /* Autotune cache: save / load (text, one line per shape key, keyed also by
  * GPU name, SM count and library version) and clear. */

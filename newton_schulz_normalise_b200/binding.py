@@ -62,7 +62,7 @@ def _load() -> ctypes.CDLL:
         "dmuon_step": (I, [PP, PP, PP, PI64, I, F, F, F, I, P]),
         "dmuon_step_ex": (I, [PP, PP, PP, PI64, I, F, F, F, I, ctypes.POINTER(Options), P]),
         "dmuon_compute_update": (I, [PP, PP, PI64, I, F, I, ctypes.POINTER(Options), PP, P]),
-        "dmuon_gemm_bf16": (I, [P, I64, I64, P, I64, I64, I, P, I64, I64, P, I64, I64, I, I, I, I, F, F, I, P]),
+        "dmuon_gemm_bf16": (I, [P, I64, I64, P, I64, I64, I, P, I64, I64, P, I64, I64, I, I, I, I, F, F, I, I, P]),
         "dmuon_cache_save": (I, [ctypes.c_char_p]),
         "dmuon_cache_load": (I, [ctypes.c_char_p]),
         "dmuon_cache_clear": (None, []),
@@ -194,8 +194,9 @@ def dmuon_compute_update_noalloc(grad, momentum, out, mu, ns_steps=5, opts: Opti
                                                    _stream(stream)))
 
 
-def dmuon_gemm_bf16(A, B, D, alpha=1.0, beta=0.0, C=None, b_kmajor=True, bn=0, stream=None):
-    """D = alpha * A @ op(B) + beta * C on 2-D or 3-D (batched) bf16 tensors."""
+def dmuon_gemm_bf16(A, B, D, alpha=1.0, beta=0.0, C=None, b_kmajor=True, tile=0, sym=False, stream=None):
+    """D = alpha * A @ op(B) + beta * C on 2-D or 3-D (batched) bf16 tensors.
+    tile: 128 / 256 (one CTA per 128 x tile), 512 (CTA pair per 256 x 256)."""
     def geom(t):
         if t.dim() == 2:
             return 1, t.shape[0], t.shape[1], t.stride(0), t.shape[0] * t.stride(0)
@@ -209,7 +210,8 @@ def dmuon_gemm_bf16(A, B, D, alpha=1.0, beta=0.0, C=None, b_kmajor=True, bn=0, s
         _, _, _, ldc, sc = geom(C)
     return _check(lib.dmuon_gemm_bf16(A.data_ptr(), lda, sa, B.data_ptr(), ldb, sb, int(b_kmajor),
                                       C.data_ptr() if C is not None else None, ldc, sc,
-                                      D.data_ptr(), ldd, sd, M, N, K, batch, alpha, beta, bn, _stream(stream)))
+                                      D.data_ptr(), ldd, sd, M, N, K, batch, alpha, beta, tile, int(sym),
+                                      _stream(stream)))
 
 
 def dmuon_cache_save(path: str):

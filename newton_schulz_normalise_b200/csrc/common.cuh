@@ -90,6 +90,29 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
+// 3-D tiled store from CTA shared memory (bulk async group of this thread).
+// Elements of the box outside the tensor are not written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(m),
+               "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy (TMA) reads of them.
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
@@ -146,6 +169,68 @@ __device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// ---------------------------------------------------------------- CTA pairs (cta_group::2)
+// A cluster of two CTAs on neighbouring SMs shares one 256-row MMA: the
+// leader (rank 0) issues it, each CTA supplies half of A and half of B from
+// its own shared memory and holds half of the accumulator in its own TMEM.
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Shared-memory address of the same object in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t out;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(addr), "r"(rank));
+  return out;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void tmem_alloc2(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish2() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on the mbarrier at `bar`'s offset in every CTA of `mask` once the
+// pair's MMAs issued so far are done.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+// 3-D tiled load into this CTA's shared memory whose completion is counted
+// on an mbarrier that may live in the peer CTA (cluster address).  No
+// multicast: each CTA fetches its own half.
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster, int x,
+                                                 int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(m), "r"(bar_cluster), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
 // Shared-memory matrix descriptor for a 128-byte-swizzled bf16 tile.
 //   K-major operand (rows of 64 elements = 128 B along K): lbo unused (16),
 //     sbo = 1024 (distance between 8-row groups).
@@ -194,6 +279,9 @@ struct Epilogue {
   int transposed;                // the iterate is the transpose of the stored matrix
   long long ldw;                 // row length of the stored (original) matrix
   float decay, lr_scale;         // W <- decay*W - lr_scale*O
+  int sym;                       // EPI_STORE of a symmetric M x M result: only the blocks on
+                                 // and above the block diagonal run; blocks above it are
+                                 // also stored mirrored (see the tensor-core kernels)
 };
 
 __device__ __forceinline__ float load_elem(const void* p, long long i, int is_f32) {
@@ -209,10 +297,12 @@ __device__ __forceinline__ void store_elem(void* p, long long i, float v, int is
 
 // Applies the epilogue to `cnt` (<= 32) consecutive columns col..col+cnt-1 of
 // row `row` of matrix `l`; v[] holds the fp32 accumulators.  M, N bound the
-// valid region.  Vector paths need 16-byte aligned rows (checked).
+// valid region.  Vector paths need 16-byte aligned rows (checked).  With
+// `mirror` (EPI_STORE of a symmetric result) every element is also stored at
+// its transposed position.
 template <int CNT>
 __device__ __forceinline__ void epilogue_row(const Epilogue& e, int l, int row, int col, const float (&v)[CNT],
-                                             int M, int N) {
+                                             int M, int N, bool mirror = false) {
   if (row >= M) return;
   float alpha = e.alpha, beta = e.beta;
   if (e.alpha_vec) alpha *= e.alpha_vec[l];
@@ -252,6 +342,14 @@ __device__ __forceinline__ void epilogue_row(const Epilogue& e, int l, int row, 
   // ---- output
   if (e.mode == EPI_STORE) {
     const long long dbase = static_cast<long long>(l) * e.sd + static_cast<long long>(row) * e.ldd + col;
+    if (mirror) {
+      // (c, row): lanes hold consecutive rows, so each c is one contiguous
+      // segment across the warp
+      const long long mbase = static_cast<long long>(l) * e.sd + row;
+#pragma unroll
+      for (int j = 0; j < CNT; ++j)
+        if (col + j < N) store_elem(e.D, mbase + static_cast<long long>(col + j) * e.ldd, o[j], e.d_f32);
+    }
     if (!e.d_f32 && full && (CNT % 8 == 0) && ((dbase & 7) == 0)) {
       uint4* dp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(e.D) + dbase);
 #pragma unroll

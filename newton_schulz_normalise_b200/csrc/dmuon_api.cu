@@ -195,7 +195,7 @@ int ensure_ws(DeviceCtx& c, size_t bytes, cudaStream_t s) {
 // ------------------------------------------------------------------ plans
 struct Plan {
   int variant = DMUON_VARIANT_DIRECT;
-  int bn = 256;
+  int tile = 256;        // 128 / 256: one CTA per 128 x tile output tile; 512: CTA pair, 256 x 256
   double cost_ms = 0.0;  // measured for one chunk of `chunk` matrices
 };
 
@@ -309,20 +309,25 @@ T* at(const Chunk& ch, size_t off) {
 
 // One GEMM of the NS recursion.  A: M x K rows (ld lda), B: K-major (N x K)
 // or MN-major (K x N).  Dispatches to tensor cores (bf16) or SIMT (fp32).
-int gemm(DeviceCtx& c, const Geo& g, int cnt, bool f32, int bn, const void* A, long long lda, long long sa,
+// sym: the M x M result is symmetric; the tensor-core kernels compute only the
+// tiles that meet the upper triangle and mirror them (FLOPs counted for the
+// computed tiles only).
+int gemm(DeviceCtx& c, int cnt, bool f32, int tile, bool sym, const void* A, long long lda, long long sa,
          const void* B, long long ldb, long long sb, bool b_kmajor, int M, int N, int K, const Epilogue& e,
          cudaStream_t s) {
-  const double flops = 2.0 * M * N * static_cast<double>(K) * cnt;
   cudaError_t err;
   if (!f32) {
-    TcGemm t{A, lda, sa, B, ldb, sb, b_kmajor, M, N, K, cnt, bn, e};
+    const long long tiles = tc_gemm_tiles(M, N, cnt, tile, sym);
+    const long long dense = tc_gemm_tiles(M, N, cnt, tile, false);
+    const double flops = 2.0 * M * N * static_cast<double>(K) * cnt * static_cast<double>(tiles) / dense;
+    TcGemm t{A, lda, sa, B, ldb, sb, b_kmajor, M, N, K, cnt, tile, sym, e};
     err = launch_k(KIND_TC_GEMM, flops, 0.0, s, [&] { return launch_tc_gemm(t, s, c.err_dev, c.num_sms); });
   } else {
+    const double flops = 2.0 * M * N * static_cast<double>(K) * cnt;
     SimtGemm t{static_cast<const float*>(A), lda, sa, static_cast<const float*>(B), ldb, sb, b_kmajor, M, N, K, cnt, e};
     err = launch_k(KIND_SIMT_GEMM, flops, 0.0, s, [&] { return launch_simt_gemm(t, s); });
   }
   if (err != cudaSuccess) return fail(DMUON_ERR_CUDA, "gemm %dx%dx%d (batch %d) launch failed: %s", M, N, K, cnt, cudaGetErrorString(err));
-  (void)g;
   return DMUON_OK;
 }
 
@@ -371,7 +376,7 @@ int run_momentum(DeviceCtx& c, const Chunk& ch, bool f32, bool g_f32, const Hype
 
 // Newton-Schulz on X0 (unnormalised U, scale s folded into the first
 // products), finishing with `fin` (apply / out / store) on the result.
-int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int bn, const Hyper& h, const Epilogue& fin_in,
+int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const Hyper& h, const Epilogue& fin_in,
            int cnt, cudaStream_t s) {
   const Geo& g = *ch.g;
   const int m = g.m, n = g.n;
@@ -403,7 +408,7 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int bn, const H
     void* T = at<void>(ch, ch.L.T);
     void* Q[2] = {at<void>(ch, ch.L.Q0), at<void>(ch, ch.L.Q1)};
     // G = s^2 U U^T  (A_0): both operands are rows of U (K-major)
-    rc = gemm(c, g, cnt, f32, bn, X0, g.ldx, sx, X0, g.ldx, sx, true, m, m, n, store_epi(A, g.ldm, sq, f32, 1.f, s2v), s);
+    rc = gemm(c, cnt, f32, tile, true, X0, g.ldx, sx, X0, g.ldx, sx, true, m, m, n, store_epi(A, g.ldm, sq, f32, 1.f, s2v), s);
     if (rc) return rc;
     int qi = 0;
     for (int k = 0; k < h.steps; ++k) {
@@ -415,19 +420,19 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int bn, const H
       ep.sc = sq;
       ep.beta = h.b;
       ep.diag = h.a;
-      rc = gemm(c, g, cnt, f32, bn, A, g.ldm, sq, A, g.ldm, sq, false, m, m, m, ep, s);
+      rc = gemm(c, cnt, f32, tile, true, A, g.ldm, sq, A, g.ldm, sq, false, m, m, m, ep, s);
       if (rc) return rc;
       if (k > 0) {  // Q_{k+1} = P_k Q_k
-        rc = gemm(c, g, cnt, f32, bn, Pk, g.ldm, sq, Q[qi], g.ldm, sq, false, m, m, m,
+        rc = gemm(c, cnt, f32, tile, true, Pk, g.ldm, sq, Q[qi], g.ldm, sq, false, m, m, m,
                   store_epi(Q[qi ^ 1], g.ldm, sq, f32, 1.f, nullptr), s);
         if (rc) return rc;
         qi ^= 1;
       }
       if (k < h.steps - 1) {  // A_{k+1} = P_k A_k P_k
-        rc = gemm(c, g, cnt, f32, bn, Pk, g.ldm, sq, A, g.ldm, sq, false, m, m, m,
+        rc = gemm(c, cnt, f32, tile, true, Pk, g.ldm, sq, A, g.ldm, sq, false, m, m, m,
                   store_epi(T, g.ldm, sq, f32, 1.f, nullptr), s);
         if (rc) return rc;
-        rc = gemm(c, g, cnt, f32, bn, T, g.ldm, sq, Pk, g.ldm, sq, false, m, m, m,
+        rc = gemm(c, cnt, f32, tile, true, T, g.ldm, sq, Pk, g.ldm, sq, false, m, m, m,
                   store_epi(A, g.ldm, sq, f32, 1.f, nullptr), s);
         if (rc) return rc;
       }
@@ -437,7 +442,7 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int bn, const H
     fin.alpha_vec = sv;
     fin.beta = 0.f;
     fin.C = nullptr;
-    return gemm(c, g, cnt, f32, bn, Q[qi], g.ldm, sq, X0, g.ldx, sx, false, m, n, m, fin, s);
+    return gemm(c, cnt, f32, tile, false, Q[qi], g.ldm, sq, X0, g.ldx, sx, false, m, n, m, fin, s);
   }
   // ---------------- direct form
   void* A = at<void>(ch, ch.L.A);
@@ -448,7 +453,7 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int bn, const H
     const bool first = (k == 0);
     const bool last = (k == h.steps - 1);
     // A = X X^T  (s^2 folded in on the first step)
-    rc = gemm(c, g, cnt, f32, bn, cur, g.ldx, sx, cur, g.ldx, sx, true, m, m, n,
+    rc = gemm(c, cnt, f32, tile, true, cur, g.ldx, sx, cur, g.ldx, sx, true, m, m, n,
               store_epi(A, g.ldm, sq, f32, 1.f, first ? s2v : nullptr), s);
     if (rc) return rc;
     // Bm = c A A + b A   (right operand as stored, see the Gram form)
@@ -457,7 +462,7 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int bn, const H
     ep.ldc = g.ldm;
     ep.sc = sq;
     ep.beta = h.b;
-    rc = gemm(c, g, cnt, f32, bn, A, g.ldm, sq, A, g.ldm, sq, false, m, m, m, ep, s);
+    rc = gemm(c, cnt, f32, tile, true, A, g.ldm, sq, A, g.ldm, sq, false, m, m, m, ep, s);
     if (rc) return rc;
     // X' = Bm X + a X   (times s on the first step)
     void* nxt = bufs[k & 1];
@@ -470,7 +475,7 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int bn, const H
     eu.ldc = g.ldx;
     eu.sc = sx;
     eu.c_f32 = f32;
-    rc = gemm(c, g, cnt, f32, bn, Bm, g.ldm, sq, cur, g.ldx, sx, false, m, n, m, eu, s);
+    rc = gemm(c, cnt, f32, tile, false, Bm, g.ldm, sq, cur, g.ldx, sx, false, m, n, m, eu, s);
     if (rc) return rc;
     cur = nxt;
   }
@@ -526,11 +531,12 @@ int validate(const Request& r) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-int forced_bn() {
-  const char* b = getenv("DMUON_BN");
+// DMUON_TILE=128|256|512 restricts the autotuner to one tile shape.
+int forced_tile() {
+  const char* b = getenv("DMUON_TILE");
   if (b) {
     int v = atoi(b);
-    if (v == 128 || v == 256) return v;
+    if (v == 128 || v == 256 || v == 512) return v;
   }
   return 0;
 }
@@ -577,10 +583,10 @@ Epilogue final_epilogue(const Request& r, const Geo& g, const Chunk& ch, bool f3
   return e;
 }
 
-int time_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int bn, const Hyper& h, const Epilogue& fin,
+int time_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const Hyper& h, const Epilogue& fin,
             int cnt, cudaStream_t s, float* ms) {
   CUDA_TRY(cudaEventRecord(c.tune_a, s));
-  int rc = run_ns(c, ch, f32, variant, bn, h, fin, cnt, s);
+  int rc = run_ns(c, ch, f32, variant, tile, h, fin, cnt, s);
   if (rc) return rc;
   CUDA_TRY(cudaEventRecord(c.tune_b, s));
   CUDA_TRY(cudaEventSynchronize(c.tune_b));
@@ -591,20 +597,22 @@ int time_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int bn, const 
 
 // Chooses the plan for a group by timing candidates on the chunk's own data
 // (after the momentum kernel produced X0).  Candidates write their result
-// into scratch (Xq region reused as the output), never into the caller's
-// buffers.  Direct form with bn 256 is the accuracy reference of the gate.
+// into scratch beyond the chunk layout, never into the caller's buffers.  The
+// first candidate (direct form) is the accuracy reference of the gate.
 int autotune(DeviceCtx& c, const Chunk& ch, bool f32, const Hyper& h, int forced_variant, Plan* plan,
              cudaStream_t s) {
   const Geo& g = *ch.g;
-  std::vector<std::pair<int, int>> cands;  // (variant, bn)
-  const int fbn = forced_bn();
-  std::vector<int> bns;
+  std::vector<std::pair<int, int>> cands;  // (variant, tile)
+  const int ft = forced_tile();
+  std::vector<int> tiles;
   if (f32)
-    bns = {0};
-  else if (fbn)
-    bns = {fbn};
+    tiles = {256};  // the SIMT path has one tile shape
+  else if (ft)
+    tiles = {ft};
+  else if (g.m >= 256)
+    tiles = {512, 256, 128};
   else
-    bns = {256, 128};
+    tiles = {256, 128};
   std::vector<int> vars;
   if (forced_variant == DMUON_VARIANT_DIRECT || forced_variant == DMUON_VARIANT_GRAM)
     vars = {forced_variant};
@@ -613,14 +621,9 @@ int autotune(DeviceCtx& c, const Chunk& ch, bool f32, const Hyper& h, int forced
     if (g.n * 4 >= g.m * 5 && h.steps > 0) vars.push_back(DMUON_VARIANT_GRAM);  // n >= 1.25 m
   }
   for (int v : vars)
-    for (int b : bns) cands.push_back({v, b});
-  if (h.steps == 0) cands = {{DMUON_VARIANT_DIRECT, bns[0]}};
+    for (int t : tiles) cands.push_back({v, t});
+  if (h.steps == 0) cands = {{DMUON_VARIANT_DIRECT, tiles[0]}};
 
-  // Output of each candidate: reuse the Xp region for the reference and a
-  // second region (Xq) for the challenger; direct ping-pongs Xp/Xq itself,
-  // so candidates store their final result into the P/Q regions' space only
-  // when it fits.  Simplest safe choice: store the final result in X-sized
-  // scratch appended after the layout (`out` below).
   const int probe = ch.cnt;
   uint8_t* outbuf = ch.base + ch.L.total;  // two X-sized slots reserved by the caller
   const size_t xb = align256(static_cast<size_t>(probe) * g.x_elems() * g.esz);
@@ -631,15 +634,15 @@ int autotune(DeviceCtx& c, const Chunk& ch, bool f32, const Hyper& h, int forced
   float best = 1e30f;
   Plan bestp;
   bool have_ref = false;
-  for (auto [v, bn] : cands) {
+  for (auto [v, tile] : cands) {
     const bool is_ref = !have_ref;
     void* dst = is_ref ? ref_out : cand_out;
     Epilogue fin = store_epi(dst, g.ldx, g.x_elems(), f32, 1.f, nullptr);
     float ms = 0.f;
     // warm once (first launch of a kernel instance loads the module), then time
-    int rc = run_ns(c, ch, f32, v, bn == 0 ? 256 : bn, h, fin, probe, s);
+    int rc = run_ns(c, ch, f32, v, tile, h, fin, probe, s);
     if (rc) return rc;
-    rc = time_ns(c, ch, f32, v, bn == 0 ? 256 : bn, h, fin, probe, s, &ms);
+    rc = time_ns(c, ch, f32, v, tile, h, fin, probe, s, &ms);
     if (rc) return rc;
     bool pass = true;
     double relerr = 0.0;
@@ -654,13 +657,13 @@ int autotune(DeviceCtx& c, const Chunk& ch, bool f32, const Hyper& h, int forced
       pass = relerr <= gate_tol();
     }
     if (trace_on())
-      fprintf(stderr, "[dmuon] tune %dx%d cnt=%d variant=%d bn=%d: %.3f ms%s gate=%.2e %s\n", g.rows, g.cols, probe, v,
-              bn, ms, is_ref ? " (reference)" : "", relerr, pass ? "pass" : "REJECT");
+      fprintf(stderr, "[dmuon] tune %dx%d cnt=%d variant=%d tile=%d: %.3f ms%s gate=%.2e %s\n", g.rows, g.cols, probe,
+              v, tile, ms, is_ref ? " (reference)" : "", relerr, pass ? "pass" : "REJECT");
     have_ref = true;
     if (pass && ms < best) {
       best = ms;
       bestp.variant = v;
-      bestp.bn = bn == 0 ? 256 : bn;
+      bestp.tile = tile;
       bestp.cost_ms = ms;
     }
   }
@@ -795,12 +798,12 @@ int run_step(Request& r) {
         if (r.o.variant == DMUON_VARIANT_AUTO || !g_cache.count(key)) g_cache[key] = pl;
       }
       Epilogue fin = final_epilogue(r, g, ch, f32);
-      rc = run_ns(c, ch, f32, gr.plan.variant, gr.plan.bn, r.h, fin, ch.cnt, r.s);
+      rc = run_ns(c, ch, f32, gr.plan.variant, gr.plan.tile, r.h, fin, ch.cnt, r.s);
       if (rc) return rc;
     }
     if (trace_on())
-      fprintf(stderr, "[dmuon] group %lldx%lld x%d: variant=%d bn=%d chunk=%d cost=%.3f ms\n", gr.rows, gr.cols, total,
-              gr.plan.variant, gr.plan.bn, gr.chunk, gr.plan.cost_ms);
+      fprintf(stderr, "[dmuon] group %lldx%lld x%d: variant=%d tile=%d chunk=%d cost=%.3f ms\n", gr.rows, gr.cols,
+              total, gr.plan.variant, gr.plan.tile, gr.chunk, gr.plan.cost_ms);
   }
   CUDA_TRY(cudaEventRecord(c.last_done, r.s));
   c.has_last = true;
@@ -974,12 +977,12 @@ int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows,
   fin.transposed = g.transposed;
   fin.ldw = g.cols;
   fin.w_f32 = f32;
-  return run_ns(c, ch, f32, plan.variant, plan.bn, r.h, fin, 1, s);
+  return run_ns(c, ch, f32, plan.variant, plan.tile, r.h, fin, 1, s);
 }
 
 int dmuon_gemm_bf16(const void* A, int64_t lda, int64_t sa, const void* B, int64_t ldb, int64_t sb, int b_kmajor,
                     const void* C, int64_t ldc, int64_t sc, void* D, int64_t ldd, int64_t sd, int M, int N, int K,
-                    int batch, float alpha, float beta, int bn, void* stream) {
+                    int batch, float alpha, float beta, int tile, int sym, void* stream) {
   t_err.clear();
   if (!A || !B || !D) return fail(DMUON_ERR_INVALID, "null operand");
   if (M <= 0 || N <= 0 || K <= 0 || batch <= 0) return fail(DMUON_ERR_INVALID, "bad GEMM size");
@@ -987,7 +990,8 @@ int dmuon_gemm_bf16(const void* A, int64_t lda, int64_t sa, const void* B, int64
     return fail(DMUON_ERR_INVALID, "leading dims / batch strides must be multiples of 8");
   if (lda < K || ldd < N || (b_kmajor ? ldb < K : ldb < N) || (C && ldc < N))
     return fail(DMUON_ERR_INVALID, "leading dim smaller than the row");
-  if (bn != 0 && bn != 128 && bn != 256) return fail(DMUON_ERR_INVALID, "bn must be 0, 128 or 256");
+  if (tile != 0 && tile != 128 && tile != 256 && tile != 512) return fail(DMUON_ERR_INVALID, "tile must be 0, 128, 256 or 512");
+  if (sym && M != N) return fail(DMUON_ERR_INVALID, "sym needs M == N");
   DeviceCtx* cp = nullptr;
   int rc = get_ctx(&cp);
   if (rc) return rc;
@@ -1001,9 +1005,11 @@ int dmuon_gemm_bf16(const void* A, int64_t lda, int64_t sa, const void* B, int64
   e.D = D;
   e.ldd = ldd;
   e.sd = sd;
-  TcGemm t{A, lda, sa, B, ldb, sb, b_kmajor != 0, M, N, K, batch, bn == 0 ? 256 : bn, e};
+  const int tl = tile == 0 ? 256 : tile;
+  TcGemm t{A, lda, sa, B, ldb, sb, b_kmajor != 0, M, N, K, batch, tl, sym != 0, e};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t err = launch_k(KIND_TC_GEMM, 2.0 * M * N * static_cast<double>(K) * batch, 0.0, s,
+  const double frac = static_cast<double>(tc_gemm_tiles(M, N, batch, tl, sym != 0)) / tc_gemm_tiles(M, N, batch, tl, false);
+  cudaError_t err = launch_k(KIND_TC_GEMM, 2.0 * M * N * static_cast<double>(K) * batch * frac, 0.0, s,
                              [&] { return launch_tc_gemm(t, s, cp->err_dev, cp->num_sms); });
   if (err != cudaSuccess) return fail(DMUON_ERR_CUDA, "gemm launch: %s", cudaGetErrorString(err));
   return DMUON_OK;
@@ -1024,7 +1030,7 @@ int dmuon_cache_save(const char* path) {
   std::lock_guard<std::mutex> lk(g_cache_mu);
   for (auto& kv : g_cache)
     fprintf(f, "%lld %lld %d %d %d %d %d %.6f\n", kv.first.rows, kv.first.cols, kv.first.f32, kv.first.steps,
-            kv.first.cnt, kv.second.variant, kv.second.bn, kv.second.cost_ms);
+            kv.first.cnt, kv.second.variant, kv.second.tile, kv.second.cost_ms);
   fclose(f);
   return DMUON_OK;
 }
@@ -1052,16 +1058,16 @@ int dmuon_cache_load(const char* path) {
   }
   std::map<Key, Plan> loaded;
   long long rr, cc;
-  int f32, steps, cnt, var, bn;
+  int f32, steps, cnt, var, tile;
   double cost;
-  while (fscanf(f, "%lld %lld %d %d %d %d %d %lf", &rr, &cc, &f32, &steps, &cnt, &var, &bn, &cost) == 8) {
-    if (rr <= 0 || cc <= 0 || cnt <= 0 || (var != 1 && var != 2) || (bn != 128 && bn != 256)) {
+  while (fscanf(f, "%lld %lld %d %d %d %d %d %lf", &rr, &cc, &f32, &steps, &cnt, &var, &tile, &cost) == 8) {
+    if (rr <= 0 || cc <= 0 || cnt <= 0 || (var != 1 && var != 2) || (tile != 128 && tile != 256 && tile != 512)) {
       fclose(f);
       return fail(DMUON_ERR_INVALID, "%s: malformed entry", path);
     }
     Plan p;
     p.variant = var;
-    p.bn = bn;
+    p.tile = tile;
     p.cost_ms = cost;
     loaded[Key{rr, cc, f32, steps, cnt}] = p;
   }
@@ -1088,7 +1094,7 @@ int dmuon_cache_entry(int i, char* buf, size_t len) {
   auto it = g_cache.begin();
   std::advance(it, i);
   snprintf(buf, len, "%lld %lld %s %d %s %d %d %.4f", it->first.rows, it->first.cols, it->first.f32 ? "f32" : "bf16",
-           it->first.steps, it->second.variant == DMUON_VARIANT_GRAM ? "gram" : "direct", it->second.bn, it->first.cnt,
+           it->first.steps, it->second.variant == DMUON_VARIANT_GRAM ? "gram" : "direct", it->second.tile, it->first.cnt,
            it->second.cost_ms);
   return DMUON_OK;
 }

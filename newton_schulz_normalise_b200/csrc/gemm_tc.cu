@@ -1,26 +1,36 @@
 // gemm_tc.cu -- batched bf16 GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
 //
-// Every Newton-Schulz product of the Muon step is one launch of this kernel:
-//   A = X X^T        (both operands K-major rows of X)
-//   B = c A A + b A  (A symmetric, so A serves as its own K-major transpose)
-//   X' = B X + a X   (X is the MN-major B operand)
-// plus the Gram-space products, which have the same two operand forms.
+// Every Newton-Schulz product of the Muon step is one launch of this file's
+// kernels:
+//   A = X X^T        (both operands K-major rows of X; symmetric result)
+//   B = c A A + b A  (right operand as stored, MN-major; symmetric result)
+//   X' = B X + a X   (X is the MN-major right operand)
+// and the Gram-space products, which have the same operand forms.
 //
-// Design (one persistent CTA per SM, 256 threads, warp-specialised):
-//   warp 0 lane 0   TMA producer: 128x64 A tile + BNx64 B tile per stage,
-//                   128-byte swizzle, into a STAGES-deep ring guarded by
-//                   full/empty mbarriers.
-//   warp 1 lane 0   MMA issuer: 4 x tcgen05.mma (128 x BN x 16) per stage into
-//                   one of two TMEM accumulators (2 x BN fp32 columns), then
-//                   tcgen05.commit frees the stage / publishes the tile.
-//   warp 2          allocates and frees TMEM.
+// Two kernels, both persistent (one CTA per SM, 256 threads) and
+// warp-specialised:
+//   warp 0 lane 0   TMA producer into a ring of stages (128-byte swizzle)
+//                   guarded by full/empty mbarriers.
+//   warp 1 lane 0   MMA issuer: tcgen05.mma per 16-deep k slice into one of
+//                   two TMEM accumulators; tcgen05.commit frees the stage and
+//                   publishes a finished tile.
+//   warp 2          allocates / frees TMEM.
 //   warps 4..7      epilogue: tcgen05.ld 32 columns at a time (warp w reads
-//                   TMEM lanes 32*(w-4)..+31 = tile rows), applies
-//                   alpha*acc + beta*C (+ diag) or the fused parameter update,
-//                   stores to global, and hands the accumulator back.
-// The epilogue of tile i overlaps the main loop of tile i+1.  Every mbarrier
-// wait is bounded (2 s); on expiry the kernel records kErrTimeout in the
-// host-visible error word, every role leaves its loop and TMEM is freed.
+//                   TMEM lanes 32*(w-4)..+31 = tile rows), applies the fused
+//                   epilogue and stores; then hands the accumulator back.
+// tc_gemm_kernel:  one CTA computes a 128 x BN tile (BN = 128 or 256).
+// tc_gemm2_kernel: a cluster of two CTAs computes a 256 x 256 tile with
+//                  tcgen05.mma.cta_group::2: each CTA loads 128 rows of A and
+//                  128 rows/columns of B (32 KB per 64-deep stage instead of
+//                  48 KB for the same MMA work per SM), the leader issues the
+//                  MMA, and each CTA drains its own 128 accumulator lanes.
+// Symmetric results (sym): only blocks on or above the block diagonal run;
+// blocks above it are stored twice (as computed and mirrored).  bf16
+// results are staged per warp through shared memory and written with TMA
+// stores.
+// Every mbarrier wait is bounded (2 s); on expiry the kernel records
+// kErrTimeout in the host-visible error word, every role leaves its loop and
+// TMEM is freed.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -34,34 +44,199 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = 128 bytes = one swizzle row
 
+// Tile t of a launch -> (matrix l, tile row tm, tile column tn).  With sym
+// the result is symmetric and only blocks on or above the block diagonal run:
+// row tm holds the tiles tn >= floor(tm*bm/bn).  Tiles strictly above it
+// (tn > floor(tm*bm/bn)) are also stored mirrored; diagonal blocks are
+// computed in full and stored as they are, so every element is written once.
+__device__ __forceinline__ void decode_tile(long long t, long long per_mat, int tiles_m, int tiles_n, int bm,
+                                            int bn, bool sym, int& l, int& tm, int& tn, bool& mirror) {
+  l = static_cast<int>(t / per_mat);
+  long long u = t % per_mat;
+  mirror = false;
+  if (!sym) {
+    tm = static_cast<int>(u / tiles_n);
+    tn = static_cast<int>(u % tiles_n);
+    return;
+  }
+  for (tm = 0; tm < tiles_m; ++tm) {
+    const int first = (tm * bm) / bn;
+    const int cnt = tiles_n - first;
+    if (u < cnt) {
+      tn = first + static_cast<int>(u);
+      mirror = tn > first;
+      return;
+    }
+    u -= cnt;
+  }
+  tm = tiles_m - 1;  // not reached for t < per_mat * batch
+  tn = tiles_n - 1;
+}
+
+// ---------------------------------------------------------------- staged epilogue
+// EPI_STORE with a bf16 result goes through shared memory, one warp at a
+// time (no barrier between the four epilogue warps).  Warp w owns rows
+// 32w..32w+31 of the CTA's 128-row block and walks the tile in 32-column
+// chunks through a ring of three 32 x 32 buffers (64-byte swizzle, conflict
+// free for one row per lane):
+//   lane 0 TMA-loads the C addend of the next chunk into the ring,
+//   each lane reads its row of C, forms alpha*acc + beta*C (+ diag) and
+//   writes the bf16 result back in place, lane 0 TMA-stores the 32 x 32 box;
+//   for a mirrored tile the transposed box goes through a second pair of
+//   buffers to the mirrored position.
+// A buffer is refilled only after the store issued from it has read it
+// (bulk_wait_read).  One bulk group per chunk keeps that accounting exact.
+constexpr int CH = 32;                        // columns per chunk
+constexpr int WBOX = 32 * CH * 2;             // one 32 x 32 bf16 box, 2 KB
+constexpr int NRING = 3;                      // C / result ring per warp
+constexpr int WARP_STG = (NRING + 2) * WBOX;  // + 2 mirror buffers
+constexpr int STG_TOTAL = 4 * WARP_STG;       // 40 KB
+constexpr int NCBAR = 4 * NRING;              // one mbarrier per ring buffer
+
+struct StageState {
+  uint32_t it = 0;      // chunks processed by this warp (ring position)
+  uint32_t phases = 0;  // parity bit per ring buffer's mbarrier
+};
+
+// Issues the TMA load of the C addend of a tile's first chunk, before the
+// epilogue waits for the tile's accumulator, so the load overlaps the MMAs.
+__device__ __forceinline__ void stage_first_c(const Epilogue& e, const CUtensorMap* tmC, uint8_t* wstg, uint64_t* cbar,
+                                              int l, int row0w, int col0, int lane, const StageState& st) {
+  const float beta = e.beta * (e.beta_vec ? e.beta_vec[l] : 1.f);
+  if (e.C == nullptr || beta == 0.f || lane != 0) return;
+  bulk_wait_read<1>();  // the ring slot's previous store (three chunks back) has read it
+  const uint32_t b = st.it % NRING;
+  mbar_arrive_expect_tx(&cbar[b], WBOX);
+  tma_load_3d(wstg + b * WBOX, tmC, &cbar[b], col0, row0w, l);
+}
+
+template <int BN>
+__device__ __forceinline__ void store_tile_staged(const Epilogue& e, const CUtensorMap* tmC, const CUtensorMap* tmD,
+                                                  const CUtensorMap* tmDm, uint8_t* wstg, uint64_t* cbar,
+                                                  uint32_t tbase, int l, int row0w, int col0, int M, int N,
+                                                  bool mirror, int lane, StageState& st, volatile int* abort) {
+  float alpha = e.alpha, beta = e.beta;
+  if (e.alpha_vec) alpha *= e.alpha_vec[l];
+  if (e.beta_vec) beta *= e.beta_vec[l];
+  const bool has_c = e.C != nullptr && beta != 0.f;
+  const int row = row0w + lane;
+  constexpr int NCH = BN / CH;
+  int nlive = 0;  // chunks of this tile inside the result
+  while (nlive < NCH && col0 + nlive * CH < N) ++nlive;
+  // (the C of the tile's first chunk was issued by stage_first_c; later
+  // chunks are fetched one ahead)
+#pragma unroll 1
+  for (int i = 0; i < NCH; ++i) {
+    const int col = col0 + i * CH;
+    const uint32_t b = st.it % NRING;
+    uint8_t* buf = wstg + b * WBOX;
+    uint8_t* mbuf = wstg + (NRING + (st.it & 1)) * WBOX;
+    const bool live = i < nlive;
+    if (lane == 0) {
+      bulk_wait_read<1>();  // stores older than the previous chunk's have read their buffers
+      if (has_c && i + 1 < nlive) {
+        const uint32_t bn = (st.it + 1) % NRING;
+        mbar_arrive_expect_tx(&cbar[bn], WBOX);
+        tma_load_3d(wstg + bn * WBOX, tmC, &cbar[bn], col + CH, row0w, l);
+      }
+    }
+    __syncwarp();
+    float v[32];
+    tmem_ld_32cols(tbase + i * CH, v);  // warp-collective
+    if (live) {
+      if (has_c) {
+        mbar_wait(&cbar[b], (st.phases >> b) & 1, abort);
+        st.phases ^= 1u << b;
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4* slot = reinterpret_cast<uint4*>(buf + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4));
+        float o[8];
+        if (has_c) {
+          const uint4 cu = *slot;
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&cu);
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float2 f = __bfloat1622float2(h[t]);
+            o[2 * t] = alpha * v[q * 8 + 2 * t] + beta * f.x;
+            o[2 * t + 1] = alpha * v[q * 8 + 2 * t + 1] + beta * f.y;
+          }
+        } else {
+#pragma unroll
+          for (int t = 0; t < 8; ++t) o[t] = alpha * v[q * 8 + t];
+        }
+        if (e.diag != 0.f) {
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            if (col + q * 8 + t == row) o[t] += e.diag;
+        }
+        uint4 u;
+        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) h[t] = __floats2bfloat162_rn(o[2 * t], o[2 * t + 1]);
+        *slot = u;
+        if (mirror) {
+          __nv_bfloat16* mb = reinterpret_cast<__nv_bfloat16*>(mbuf);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) mb[(q * 8 + t) * 32 + lane] = __float2bfloat16_rn(o[t]);
+        }
+      }
+    }
+    fence_proxy_async();
+    __syncwarp();
+    if (lane == 0) {
+      if (live) {
+        tma_store_3d(tmD, buf, col, row0w, l);
+        if (mirror) tma_store_3d(tmDm, mbuf, row0w, col, l);
+      }
+      bulk_commit();
+    }
+    ++st.it;
+  }
+}
+
+long long tiles_per_matrix(int M, int N, int bm, int bn, bool sym) {
+  const int tm = (M + bm - 1) / bm, tn = (N + bn - 1) / bn;
+  if (!sym) return static_cast<long long>(tm) * tn;
+  long long s = 0;
+  for (int i = 0; i < tm; ++i) s += tn - (i * bm) / bn;
+  return s;
+}
+
 template <int BN>
 struct TcCfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int STAGES = BN == 256 ? 3 : 5;
   static constexpr int TMEM_COLS = 2 * BN;  // two accumulators
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + STG_TOTAL + 1024 /*align*/ + 256 /*barriers*/;
 };
 
+// ============================================================== one CTA per tile
 template <int BN, bool B_MN>
 __global__ void __launch_bounds__(256, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const Epilogue epi, int M, int N, int K, int batch, int* err) {
+                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
+                   const __grid_constant__ CUtensorMap tmDm, const Epilogue epi, int M, int N, int K, int batch,
+                   int sym, long long per_mat, int staged, int* err) {
   using C = TcCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* stg = smem + C::STAGES * C::STAGE_BYTES;  // 1024-aligned staging for the epilogue
+  uint64_t* full = reinterpret_cast<uint64_t*>(stg + STG_TOTAL);
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* cbar = tempty + 2;  // NCBAR: C loads of the staged epilogue
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cbar + NCBAR);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
+    for (int i = 0; i < NCBAR; ++i) mbar_init(&cbar[i], 1);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -89,17 +264,17 @@ __global__ void __launch_bounds__(256, 1)
   const int tiles_m = (M + BM - 1) / BM;
   const int tiles_n = (N + BN - 1) / BN;
   const int num_kb = (K + BK - 1) / BK;
-  const long long tiles_per_mat = static_cast<long long>(tiles_m) * tiles_n;
-  const long long total = tiles_per_mat * batch;
+  const long long total = per_mat * batch;
+  const bool sy = sym != 0;
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------ TMA producer
     int stage = 0;
     uint32_t phase = 0;
     for (long long t = blockIdx.x; t < total && !*abort; t += gridDim.x) {
-      const int l = static_cast<int>(t / tiles_per_mat);
-      const int rem = static_cast<int>(t % tiles_per_mat);
-      const int tm = rem / tiles_n, tn = rem % tiles_n;
+      int l, tm, tn;
+      bool mir;
+      decode_tile(t, per_mat, tiles_m, tiles_n, BM, BN, sy, l, tm, tn, mir);
       for (int kb = 0; kb < num_kb; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1, abort)) break;
         uint8_t* sa = smem + stage * C::STAGE_BYTES;
@@ -117,6 +292,14 @@ __global__ void __launch_bounds__(256, 1)
           stage = 0;
           phase ^= 1;
         }
+      }
+    }
+    // drain: the last commits on every stage have arrived before the CTA exits
+    for (int i = 0; i < C::STAGES && !*abort; ++i) {
+      if (!mbar_wait(&empty[stage], phase ^ 1, abort)) break;
+      if (++stage == C::STAGES) {
+        stage = 0;
+        phase ^= 1;
       }
     }
   } else if (warp == 1 && lane == 0) {
@@ -164,10 +347,13 @@ __global__ void __launch_bounds__(256, 1)
     const int ew = warp - 4;
     int acc = 0;
     uint32_t acc_phase = 0;
+    StageState st;
+    uint8_t* wstg = stg + ew * WARP_STG;
     for (long long t = blockIdx.x; t < total; t += gridDim.x) {
-      const int l = static_cast<int>(t / tiles_per_mat);
-      const int rem = static_cast<int>(t % tiles_per_mat);
-      const int tm = rem / tiles_n, tn = rem % tiles_n;
+      int l, tm, tn;
+      bool mir;
+      decode_tile(t, per_mat, tiles_m, tiles_n, BM, BN, sy, l, tm, tn, mir);
+      if (staged) stage_first_c(epi, &tmC, wstg, cbar + ew * NRING, l, tm * BM + ew * 32, tn * BN, lane, st);
       // every lane observes the barrier; the vote reconverges the warp before
       // the warp-collective tcgen05.ld and makes an abort warp-uniform
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, abort));
@@ -175,12 +361,17 @@ __global__ void __launch_bounds__(256, 1)
       tc_fence_after();
       const int row = tm * BM + ew * 32 + lane;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + acc * BN;
+      if (staged) {
+        store_tile_staged<BN>(epi, &tmC, &tmD, &tmDm, wstg, cbar + ew * NRING, tbase, l, tm * BM + ew * 32, tn * BN,
+                              M, N, mir, lane, st, abort);
+      } else {
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        const int col = tn * BN + c0;
-        float v[32];
-        tmem_ld_32cols(tbase + c0, v);  // warp-collective: all lanes participate
-        if (col < N) epilogue_row<32>(epi, l, row, col, v, M, N);
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          const int col = tn * BN + c0;
+          float v[32];
+          tmem_ld_32cols(tbase + c0, v);  // warp-collective: all lanes participate
+          if (col < N) epilogue_row<32>(epi, l, row, col, v, M, N, mir);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -192,11 +383,206 @@ __global__ void __launch_bounds__(256, 1)
     }
   }
 
+  if (warp >= 4 && lane == 0) bulk_wait<0>();  // each warp's staged stores complete before the CTA exits
   __syncthreads();
   if (*abort && threadIdx.x == 0 && err) *reinterpret_cast<volatile int*>(err) = kErrTimeout;
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ============================================================== CTA pair per 256 x 256 tile
+constexpr int P_BM = 256;                       // tile rows (128 per CTA)
+constexpr int P_BN = 256;                       // tile columns (128 per CTA's B half)
+constexpr int P_A_BYTES = BM * BK * 2;          // 16 KB
+constexpr int P_B_BYTES = (P_BN / 2) * BK * 2;  // 16 KB
+constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;
+constexpr int P_STAGES = 5;
+constexpr int P_TMEM_COLS = 2 * P_BN;  // two 256-column accumulators = all 512 columns
+constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + STG_TOTAL + 1024 + 256;
+
+template <bool B_MN>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
+    tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
+                    const __grid_constant__ CUtensorMap tmDm, const Epilogue epi, int M, int N, int K, int batch,
+                    int sym, long long per_mat, int staged, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stg = smem + P_STAGES * P_STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(stg + STG_TOTAL);
+  uint64_t* empty = full + P_STAGES;
+  uint64_t* tfull = empty + P_STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* cbar = tempty + 2;  // NCBAR: C loads of the staged epilogue
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cbar + NCBAR);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();  // 0 = leader (issues the MMA)
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NCBAR; ++i) mbar_init(&cbar[i], 1);
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(&full[s], 1);   // used in the leader only: its arrive_expect_tx
+      mbar_init(&empty[s], 1);  // one multicast commit per phase, in both CTAs
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);   // multicast commit, both CTAs
+      mbar_init(&tempty[a], 8);  // leader's: 4 epilogue warps x 2 CTAs
+    }
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 2) {
+    tmem_alloc2(tmem_slot, P_TMEM_COLS);
+    tmem_relinquish2();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers initialised before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int tiles_m = (M + P_BM - 1) / P_BM;
+  const int tiles_n = (N + P_BN - 1) / P_BN;
+  const int num_kb = (K + BK - 1) / BK;
+  const long long total = per_mat * batch;
+  const bool sy = sym != 0;
+  const int pair = blockIdx.x >> 1;
+  const int npairs = gridDim.x >> 1;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------ TMA producer (both CTAs)
+    int stage = 0;
+    uint32_t phase = 0;
+    for (long long t = pair; t < total && !*abort; t += npairs) {
+      int l, tm, tn;
+      bool mir;
+      decode_tile(t, per_mat, tiles_m, tiles_n, P_BM, P_BN, sy, l, tm, tn, mir);
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort)) break;
+        uint8_t* sa = smem + stage * P_STAGE_BYTES;
+        uint8_t* sb = sa + P_A_BYTES;
+        const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
+        if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * P_STAGE_BYTES);
+        tma_load_3d_pair(sa, &tmA, fbar, kb * BK, tm * P_BM + static_cast<int>(rank) * BM, l);
+        const int n0 = tn * P_BN + static_cast<int>(rank) * (P_BN / 2);
+        if (B_MN) {
+#pragma unroll
+          for (int j = 0; j < P_BN / 2 / 64; ++j)
+            tma_load_3d_pair(sb + j * (BK * 128), &tmB, fbar, n0 + j * 64, kb * BK, l);
+        } else {
+          tma_load_3d_pair(sb, &tmB, fbar, kb * BK, n0, l);
+        }
+        if (++stage == P_STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    for (int i = 0; i < P_STAGES && !*abort; ++i) {  // drain the last commits
+      if (!mbar_wait(&empty[stage], phase ^ 1, abort)) break;
+      if (++stage == P_STAGES) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ------------------------------------------------ MMA issuer (leader)
+    constexpr uint32_t IDESC = idesc_bf16_f32(P_BM, P_BN, B_MN);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (long long t = pair; t < total && !*abort; t += npairs) {
+      if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * P_BN;
+      bool ok = true;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait(&full[stage], phase, abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + stage * P_STAGE_BYTES);
+        const uint32_t sb = sa + P_A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t adesc = smem_desc_sw128(sa + kk * 32, 16, 1024);
+          const uint64_t bdesc =
+              B_MN ? smem_desc_sw128(sb + kk * 16 * 128, BK * 128, 1024) : smem_desc_sw128(sb + kk * 32, 16, 1024);
+          umma_bf16_pair(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+        }
+        umma_commit_pair(&empty[stage], 0x3);
+        if (++stage == P_STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) break;
+      umma_commit_pair(&tfull[acc], 0x3);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------ epilogue (both CTAs)
+    const int ew = warp - 4;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    StageState st;
+    uint8_t* wstg = stg + ew * WARP_STG;
+    for (long long t = pair; t < total; t += npairs) {
+      int l, tm, tn;
+      bool mir;
+      decode_tile(t, per_mat, tiles_m, tiles_n, P_BM, P_BN, sy, l, tm, tn, mir);
+      if (staged)
+        stage_first_c(epi, &tmC, wstg, cbar + ew * NRING, l, tm * P_BM + static_cast<int>(rank) * BM + ew * 32,
+                      tn * P_BN, lane, st);
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, abort));
+      if (!ok) break;
+      tc_fence_after();
+      const int row0 = tm * P_BM + static_cast<int>(rank) * BM;
+      const int row = row0 + ew * 32 + lane;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + acc * P_BN;
+      if (staged) {
+        store_tile_staged<P_BN>(epi, &tmC, &tmD, &tmDm, wstg, cbar + ew * NRING, tbase, l, row0 + ew * 32,
+                                tn * P_BN, M, N, mir, lane, st, abort);
+      } else {
+#pragma unroll 1
+        for (int c0 = 0; c0 < P_BN; c0 += 32) {
+          const int col = tn * P_BN + c0;
+          float v[32];
+          tmem_ld_32cols(tbase + c0, v);
+          if (col < N) epilogue_row<32>(epi, l, row, col, v, M, N, mir);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[acc]), 0));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  if (warp >= 4 && lane == 0) bulk_wait<0>();  // each warp's staged stores complete before the CTA exits
+  __syncthreads();
+  cluster_sync();  // no CTA leaves while its peer may still signal its barriers
+  if (*abort && threadIdx.x == 0 && err) *reinterpret_cast<volatile int*>(err) = kErrTimeout;
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc2(tmem_base, P_TMEM_COLS);
   }
 }
 
@@ -215,9 +601,10 @@ cudaError_t get_encode() {
   return g_encode ? cudaSuccess : cudaErrorNotSupported;
 }
 
-// 3-D bf16 tensor map {inner, outer, batch} with 128-byte swizzle.
+// 3-D bf16 tensor map {inner, outer, batch}.
 bool make_map(CUtensorMap* m, const void* base, long long inner, long long outer, int batch, long long ld,
-              long long bstride, int box_inner, int box_outer) {
+              long long bstride, int box_inner, int box_outer,
+              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer),
                         static_cast<cuuint64_t>(batch)};
   long long bs = batch > 1 ? bstride : ld * outer;
@@ -225,13 +612,29 @@ bool make_map(CUtensorMap* m, const void* base, long long inner, long long outer
   cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
+// Maps of the staged epilogue: 32 x 32 boxes of C (load) and of D (store),
+// 64-byte swizzle to match the staging layout, and the mirrored 32 x 32 box
+// of D without swizzle.  Returns false when the result cannot take the staged
+// path (the epilogue then stores from registers).
+bool make_stage_maps(const TcGemm& g, CUtensorMap* mc, CUtensorMap* md, CUtensorMap* mm) {
+  const Epilogue& e = g.epi;
+  if (e.mode != EPI_STORE || e.d_f32 || !e.D) return false;
+  if ((reinterpret_cast<uintptr_t>(e.D) & 15) || (e.ldd & 7) || (g.batch > 1 && (e.sd & 7))) return false;
+  if (e.C && (e.c_f32 || (reinterpret_cast<uintptr_t>(e.C) & 15) || (e.ldc & 7) || (g.batch > 1 && (e.sc & 7))))
+    return false;
+  if (!make_map(md, e.D, g.N, g.M, g.batch, e.ldd, e.sd, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return false;
+  if (!make_map(mm, e.D, g.N, g.M, g.batch, e.ldd, e.sd, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE)) return false;
+  if (e.C && !make_map(mc, e.C, g.N, g.M, g.batch, e.ldc, e.sc, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return false;
+  return true;
+}
+
 template <int BN, bool B_MN>
-cudaError_t launch_impl(const TcGemm& g, cudaStream_t s, int* dev_err, int num_sms) {
+cudaError_t launch_one(const TcGemm& g, cudaStream_t s, int* dev_err, int num_sms) {
   using C = TcCfg<BN>;
   static std::once_flag attr_once;
   static cudaError_t attr_err = cudaSuccess;
@@ -245,26 +648,81 @@ cudaError_t launch_impl(const TcGemm& g, cudaStream_t s, int* dev_err, int num_s
   bool ok = B_MN ? make_map(&mb, g.B, g.N, g.K, g.batch, g.ldb, g.sb, 64, BK)
                  : make_map(&mb, g.B, g.K, g.N, g.batch, g.ldb, g.sb, BK, BN);
   if (!ok) return cudaErrorInvalidValue;
-  const long long tiles =
-      static_cast<long long>((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN) * static_cast<long long>(g.batch);
+  CUtensorMap mc = ma, md = ma, mm = ma;
+  const int staged = make_stage_maps(g, &mc, &md, &mm) ? 1 : 0;
+  const long long per_mat = tiles_per_matrix(g.M, g.N, BM, BN, g.sym);
+  const long long tiles = per_mat * g.batch;
   const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-  tc_gemm_kernel<BN, B_MN><<<grid, 256, C::SMEM_BYTES, s>>>(ma, mb, g.epi, g.M, g.N, g.K, g.batch, dev_err);
+  tc_gemm_kernel<BN, B_MN><<<grid, 256, C::SMEM_BYTES, s>>>(ma, mb, mc, md, mm, g.epi, g.M, g.N, g.K, g.batch,
+                                                            g.sym ? 1 : 0, per_mat, staged, dev_err);
+  return cudaGetLastError();
+}
+
+template <bool B_MN>
+cudaError_t launch_pair(const TcGemm& g, cudaStream_t s, int* dev_err, int num_sms) {
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  static int max_clusters = 0;
+  std::call_once(attr_once, [num_sms] {
+    attr_err = cudaFuncSetAttribute(tc_gemm2_kernel<B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    P_SMEM_BYTES);
+    if (attr_err != cudaSuccess) return;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (num_sms / 2));
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = P_SMEM_BYTES;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&max_clusters, tc_gemm2_kernel<B_MN>, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      max_clusters = num_sms / 2;
+    }
+    if (max_clusters <= 0) max_clusters = num_sms / 2;
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, g.A, g.K, g.M, g.batch, g.lda, g.sa, BK, BM)) return cudaErrorInvalidValue;
+  bool ok = B_MN ? make_map(&mb, g.B, g.N, g.K, g.batch, g.ldb, g.sb, 64, BK)
+                 : make_map(&mb, g.B, g.K, g.N, g.batch, g.ldb, g.sb, BK, P_BN / 2);
+  if (!ok) return cudaErrorInvalidValue;
+  CUtensorMap mc = ma, md = ma, mm = ma;
+  const int staged = make_stage_maps(g, &mc, &md, &mm) ? 1 : 0;
+  const long long per_mat = tiles_per_matrix(g.M, g.N, P_BM, P_BN, g.sym);
+  const long long tiles = per_mat * g.batch;
+  const long long pairs = tiles < max_clusters ? tiles : max_clusters;
+  tc_gemm2_kernel<B_MN><<<static_cast<int>(2 * pairs), 256, P_SMEM_BYTES, s>>>(
+      ma, mb, mc, md, mm, g.epi, g.M, g.N, g.K, g.batch, g.sym ? 1 : 0, per_mat, staged, dev_err);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+long long tc_gemm_tiles(int M, int N, int batch, int tile, bool sym) {
+  if (tile == 512) return tiles_per_matrix(M, N, P_BM, P_BN, sym) * batch;
+  return tiles_per_matrix(M, N, BM, tile == 128 ? 128 : 256, sym) * batch;
+}
+
 cudaError_t launch_tc_gemm(const TcGemm& g, cudaStream_t s, int* dev_err, int num_sms) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0 || g.batch <= 0) return cudaSuccess;
+  if (g.sym && g.M != g.N) return cudaErrorInvalidValue;
   // TMA: 16-byte aligned bases, row and batch strides multiples of 16 bytes.
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
   if (!al16(g.A) || !al16(g.B) || (g.lda & 7) || (g.ldb & 7) || (g.sa & 7) || (g.sb & 7))
     return cudaErrorMisalignedAddress;
   cudaError_t e = get_encode();
   if (e != cudaSuccess) return e;
+  TcGemm h = g;
+  h.epi.sym = g.sym ? 1 : 0;
   const bool mn = !g.b_kmajor;
-  if (g.bn == 128) return mn ? launch_impl<128, true>(g, s, dev_err, num_sms) : launch_impl<128, false>(g, s, dev_err, num_sms);
-  return mn ? launch_impl<256, true>(g, s, dev_err, num_sms) : launch_impl<256, false>(g, s, dev_err, num_sms);
+  if (g.tile == 512) return mn ? launch_pair<true>(h, s, dev_err, num_sms) : launch_pair<false>(h, s, dev_err, num_sms);
+  if (g.tile == 128)
+    return mn ? launch_one<128, true>(h, s, dev_err, num_sms) : launch_one<128, false>(h, s, dev_err, num_sms);
+  return mn ? launch_one<256, true>(h, s, dev_err, num_sms) : launch_one<256, false>(h, s, dev_err, num_sms);
 }
 
 }  // namespace dmuon

@@ -18,7 +18,8 @@ struct TcGemm {
   long long ldb, sb;
   bool b_kmajor;
   int M, N, K, batch;
-  int bn;  // tile width: 128 or 256
+  int tile;  // 128 / 256: one CTA, 128 x tile output tile; 512: CTA pair, 256 x 256
+  bool sym;  // M == N and the result is symmetric: upper-triangle tiles only, mirrored
   Epilogue epi;
 };
 
@@ -37,6 +38,8 @@ struct SimtGemm {
 enum KernelKind { KIND_TC_GEMM = 0, KIND_EW = 1, KIND_SIMT_GEMM = 2, KIND_OTHER = 3, KIND_COUNT = 4 };
 
 cudaError_t launch_tc_gemm(const TcGemm& g, cudaStream_t s, int* dev_err, int num_sms);
+// Output tiles a launch of this shape processes (symmetric skipping included).
+long long tc_gemm_tiles(int M, int N, int batch, int tile, bool sym);
 cudaError_t launch_simt_gemm(const SimtGemm& g, cudaStream_t s);
 
 // Momentum + Nesterov + per-matrix sum of squares (partials), writing the

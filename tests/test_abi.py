@@ -90,12 +90,14 @@ def test_workspace_size_is_host_only_and_monotone(dmuon_lib):
 
 def test_gemm_argument_checks(dmuon_lib):
     L = dmuon_lib
-    rc = L.lib.dmuon_gemm_bf16(None, 8, 64, None, 8, 64, 1, None, 0, 0, None, 8, 64, 8, 8, 8, 1, 1.0, 0.0, 0, None)
-    assert rc == L.DMUON_ERR_INVALID
-    rc = L.lib.dmuon_gemm_bf16(16, 12, 0, 16, 8, 0, 1, None, 0, 0, 16, 8, 0, 8, 8, 8, 1, 1.0, 0.0, 0, None)
-    assert rc == L.DMUON_ERR_INVALID  # lda not a multiple of 8
-    rc = L.lib.dmuon_gemm_bf16(16, 8, 0, 16, 8, 0, 1, None, 0, 0, 16, 8, 0, 8, 8, 8, 1, 1.0, 0.0, 96, None)
-    assert rc == L.DMUON_ERR_INVALID  # bn
+    g = L.lib.dmuon_gemm_bf16
+    assert g(None, 8, 64, None, 8, 64, 1, None, 0, 0, None, 8, 64, 8, 8, 8, 1, 1.0, 0.0, 0, 0, None) == L.DMUON_ERR_INVALID
+    # lda not a multiple of 8
+    assert g(16, 12, 0, 16, 8, 0, 1, None, 0, 0, 16, 8, 0, 8, 8, 8, 1, 1.0, 0.0, 0, 0, None) == L.DMUON_ERR_INVALID
+    # unknown tile code
+    assert g(16, 8, 0, 16, 8, 0, 1, None, 0, 0, 16, 8, 0, 8, 8, 8, 1, 1.0, 0.0, 96, 0, None) == L.DMUON_ERR_INVALID
+    # symmetric output needs a square result
+    assert g(16, 8, 0, 16, 8, 0, 1, None, 0, 0, 16, 16, 0, 8, 16, 8, 1, 1.0, 0.0, 0, 1, None) == L.DMUON_ERR_INVALID
 
 
 def test_set_workspace_alignment(dmuon_lib):
