@@ -445,8 +445,12 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
     return gemm(c, cnt, f32, tile, false, Q[qi], g.ldm, sq, X0, g.ldx, sx, false, m, n, m, fin, s);
   }
   // ---------------- direct form
+  // Per step: A = X X^T, P = c A^2 + b A + a I, X' = P X.  Folding a X into
+  // P (its identity term is the epilogue's diagonal add) leaves the X' product
+  // without an addend; in bf16 it is as accurate as adding a X in fp32 (one
+  // rounding fewer).  The scale s of the first step rides on alpha.
   void* A = at<void>(ch, ch.L.A);
-  void* Bm = at<void>(ch, ch.L.Bm);
+  void* P = at<void>(ch, ch.L.Bm);
   void* bufs[2] = {at<void>(ch, ch.L.Xp), at<void>(ch, ch.L.Xq)};
   void* cur = X0;
   for (int k = 0; k < h.steps; ++k) {
@@ -456,26 +460,24 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
     rc = gemm(c, cnt, f32, tile, true, cur, g.ldx, sx, cur, g.ldx, sx, true, m, m, n,
               store_epi(A, g.ldm, sq, f32, 1.f, first ? s2v : nullptr), s);
     if (rc) return rc;
-    // Bm = c A A + b A   (right operand as stored, see the Gram form)
-    Epilogue ep = store_epi(Bm, g.ldm, sq, f32, h.c, nullptr);
+    // P = c A A + b A + a I   (right operand as stored, see the Gram form)
+    Epilogue ep = store_epi(P, g.ldm, sq, f32, h.c, nullptr);
     ep.C = A;
     ep.ldc = g.ldm;
     ep.sc = sq;
     ep.beta = h.b;
+    ep.diag = h.a;
     rc = gemm(c, cnt, f32, tile, true, A, g.ldm, sq, A, g.ldm, sq, false, m, m, m, ep, s);
     if (rc) return rc;
-    // X' = Bm X + a X   (times s on the first step)
+    // X' = P X   (times s on the first step)
     void* nxt = bufs[k & 1];
     Epilogue eu = last ? fin : store_epi(nxt, g.ldx, sx, f32, 1.f, nullptr);
     eu.alpha = 1.f;
     eu.alpha_vec = first ? sv : nullptr;
-    eu.beta = h.a;
-    eu.beta_vec = first ? sv : nullptr;
-    eu.C = cur;
-    eu.ldc = g.ldx;
-    eu.sc = sx;
-    eu.c_f32 = f32;
-    rc = gemm(c, cnt, f32, tile, false, Bm, g.ldm, sq, cur, g.ldx, sx, false, m, n, m, eu, s);
+    eu.beta = 0.f;
+    eu.beta_vec = nullptr;
+    eu.C = nullptr;
+    rc = gemm(c, cnt, f32, tile, false, P, g.ldm, sq, cur, g.ldx, sx, false, m, n, m, eu, s);
     if (rc) return rc;
     cur = nxt;
   }
