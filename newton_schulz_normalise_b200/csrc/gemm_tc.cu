@@ -7,7 +7,7 @@
 //   X' = B X + a X   (X is the MN-major right operand)
 // and the Gram-space products, which have the same operand forms.
 //
-// Two kernels, both persistent (one CTA per SM, 256 threads) and
+// Two kernels, both persistent (one CTA per SM, 384 threads) and
 // warp-specialised:
 //   warp 0 lane 0   TMA producer into a ring of stages (128-byte swizzle)
 //                   guarded by full/empty mbarriers.
@@ -15,8 +15,9 @@
 //                   two TMEM accumulators; tcgen05.commit frees the stage and
 //                   publishes a finished tile.
 //   warp 2          allocates / frees TMEM.
-//   warps 4..7      epilogue: tcgen05.ld 32 columns at a time (warp w reads
-//                   TMEM lanes 32*(w-4)..+31 = tile rows), applies the fused
+//   warps 4..11     epilogue: tcgen05.ld 32 columns at a time (warp w reads
+//                   TMEM lanes 32*(w%4)..+31 = tile rows; the two warps of a
+//                   quarter take alternate column chunks), applies the fused
 //                   epilogue and stores; then hands the accumulator back.
 // tc_gemm_kernel:  one CTA computes a 128 x BN tile (BN = 128 or 256).
 // tc_gemm2_kernel: a cluster of two CTAs computes a 256 x 256 tile with
@@ -75,69 +76,57 @@ __device__ __forceinline__ void decode_tile(long long t, long long per_mat, int 
 
 // ---------------------------------------------------------------- staged epilogue
 // EPI_STORE with a bf16 result goes through shared memory, one warp at a
-// time (no barrier between the four epilogue warps).  Warp w owns rows
-// 32w..32w+31 of the CTA's 128-row block and walks the tile in 32-column
-// chunks through a ring of three 32 x 32 buffers (64-byte swizzle, conflict
-// free for one row per lane):
-//   lane 0 TMA-loads the C addend of the next chunk into the ring,
+// time (no barrier between the epilogue warps).  Eight epilogue warps: the
+// two warps of a TMEM lane quarter own the same 32 rows of the CTA's
+// 128-row block and take alternate 32-column chunks, so one warp's memory
+// latency overlaps its sibling's work.  Per chunk, through a ring of two
+// 32 x 32 buffers (64-byte swizzle, conflict free for one row per lane):
+//   lane 0 TMA-loads the chunk's C addend into the ring buffer,
 //   each lane reads its row of C, forms alpha*acc + beta*C (+ diag) and
 //   writes the bf16 result back in place, lane 0 TMA-stores the 32 x 32 box;
 //   for a mirrored tile the transposed box goes through a second pair of
 //   buffers to the mirrored position.
 // A buffer is refilled only after the store issued from it has read it
 // (bulk_wait_read).  One bulk group per chunk keeps that accounting exact.
+constexpr int EPI_WARPS = 8;                  // two per TMEM lane quarter, alternate chunks
+constexpr int THREADS = 128 + 32 * EPI_WARPS;  // warps 0..3: producer, MMA, TMEM, idle
 constexpr int CH = 32;                        // columns per chunk
 constexpr int WBOX = 32 * CH * 2;             // one 32 x 32 bf16 box, 2 KB
-constexpr int NRING = 3;                      // C / result ring per warp
+constexpr int NRING = 2;                      // C / result ring per warp
 constexpr int WARP_STG = (NRING + 2) * WBOX;  // + 2 mirror buffers
-constexpr int STG_TOTAL = 4 * WARP_STG;       // 40 KB
-constexpr int NCBAR = 4 * NRING;              // one mbarrier per ring buffer
+constexpr int STG_TOTAL = EPI_WARPS * WARP_STG;  // 64 KB
+constexpr int NCBAR = EPI_WARPS * NRING;      // one mbarrier per ring buffer
 
 struct StageState {
   uint32_t it = 0;      // chunks processed by this warp (ring position)
   uint32_t phases = 0;  // parity bit per ring buffer's mbarrier
 };
 
-// Issues the TMA load of the C addend of a tile's first chunk, before the
-// epilogue waits for the tile's accumulator, so the load overlaps the MMAs.
-__device__ __forceinline__ void stage_first_c(const Epilogue& e, const CUtensorMap* tmC, uint8_t* wstg, uint64_t* cbar,
-                                              int l, int row0w, int col0, int lane, const StageState& st) {
-  const float beta = e.beta * (e.beta_vec ? e.beta_vec[l] : 1.f);
-  if (e.C == nullptr || beta == 0.f || lane != 0) return;
-  bulk_wait_read<1>();  // the ring slot's previous store (three chunks back) has read it
-  const uint32_t b = st.it % NRING;
-  mbar_arrive_expect_tx(&cbar[b], WBOX);
-  tma_load_3d(wstg + b * WBOX, tmC, &cbar[b], col0, row0w, l);
-}
-
 template <int BN>
 __device__ __forceinline__ void store_tile_staged(const Epilogue& e, const CUtensorMap* tmC, const CUtensorMap* tmD,
                                                   const CUtensorMap* tmDm, uint8_t* wstg, uint64_t* cbar,
                                                   uint32_t tbase, int l, int row0w, int col0, int M, int N,
-                                                  bool mirror, int lane, StageState& st, volatile int* abort) {
+                                                  bool mirror, int lane, int half, StageState& st,
+                                                  volatile int* abort) {
   float alpha = e.alpha, beta = e.beta;
   if (e.alpha_vec) alpha *= e.alpha_vec[l];
   if (e.beta_vec) beta *= e.beta_vec[l];
   const bool has_c = e.C != nullptr && beta != 0.f;
   const int row = row0w + lane;
   constexpr int NCH = BN / CH;
-  int nlive = 0;  // chunks of this tile inside the result
-  while (nlive < NCH && col0 + nlive * CH < N) ++nlive;
-  // (the C of the tile's first chunk was issued by stage_first_c; later
-  // chunks are fetched one ahead)
+  constexpr int STRIDE = EPI_WARPS / 4;  // warps sharing this lane quarter take every STRIDE-th chunk
 #pragma unroll 1
-  for (int i = 0; i < NCH; ++i) {
+  for (int i = half; i < NCH; i += STRIDE) {
     const int col = col0 + i * CH;
     const uint32_t b = st.it % NRING;
     uint8_t* buf = wstg + b * WBOX;
     uint8_t* mbuf = wstg + (NRING + (st.it & 1)) * WBOX;
-    const bool live = i < nlive;
+    const bool live = col < N;
     if (lane == 0) {
-      bulk_wait_read<1>();  // stores older than the previous chunk's have read their buffers
-      if (has_c && i + 1 < nlive) {
-        const uint32_t bn = (st.it + 1) % NRING;
-        mbar_arrive_expect_tx(&cbar[bn], WBOX);
-        tma_load_3d(wstg + bn * WBOX, tmC, &cbar[bn], col + CH, row0w, l);
+      bulk_wait_read<1>();  // the stores issued from these buffers two chunks ago have read them
+      if (has_c && live) {
+        mbar_arrive_expect_tx(&cbar[b], WBOX);
+        tma_load_3d(buf, tmC, &cbar[b], col, row0w, l);
       }
     }
     __syncwarp();
@@ -215,7 +204,7 @@ struct TcCfg {
 
 // ============================================================== one CTA per tile
 template <int BN, bool B_MN>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
                    const __grid_constant__ CUtensorMap tmDm, const Epilogue epi, int M, int N, int K, int batch,
@@ -243,7 +232,7 @@ __global__ void __launch_bounds__(256, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);  // one arrival per epilogue warp
+      mbar_init(&tempty[a], EPI_WARPS);  // one arrival per epilogue warp
     }
     *abort = 0;
     fence_mbar_init();
@@ -344,16 +333,17 @@ __global__ void __launch_bounds__(256, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------ epilogue
-    const int ew = warp - 4;
+    const int ep = warp - 4;       // epilogue warp 0..EPI_WARPS-1
+    const int ew = warp & 3;       // TMEM lane quarter this warp may read
+    const int half = ep >> 2;      // which of the quarter's warps
     int acc = 0;
     uint32_t acc_phase = 0;
     StageState st;
-    uint8_t* wstg = stg + ew * WARP_STG;
+    uint8_t* wstg = stg + ep * WARP_STG;
     for (long long t = blockIdx.x; t < total; t += gridDim.x) {
       int l, tm, tn;
       bool mir;
       decode_tile(t, per_mat, tiles_m, tiles_n, BM, BN, sy, l, tm, tn, mir);
-      if (staged) stage_first_c(epi, &tmC, wstg, cbar + ew * NRING, l, tm * BM + ew * 32, tn * BN, lane, st);
       // every lane observes the barrier; the vote reconverges the warp before
       // the warp-collective tcgen05.ld and makes an abort warp-uniform
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, abort));
@@ -362,11 +352,11 @@ __global__ void __launch_bounds__(256, 1)
       const int row = tm * BM + ew * 32 + lane;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + acc * BN;
       if (staged) {
-        store_tile_staged<BN>(epi, &tmC, &tmD, &tmDm, wstg, cbar + ew * NRING, tbase, l, tm * BM + ew * 32, tn * BN,
-                              M, N, mir, lane, st, abort);
+        store_tile_staged<BN>(epi, &tmC, &tmD, &tmDm, wstg, cbar + ep * NRING, tbase, l, tm * BM + ew * 32, tn * BN,
+                              M, N, mir, lane, half, st, abort);
       } else {
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 32) {
+        for (int c0 = half * 32; c0 < BN; c0 += 32 * (EPI_WARPS / 4)) {
           const int col = tn * BN + c0;
           float v[32];
           tmem_ld_32cols(tbase + c0, v);  // warp-collective: all lanes participate
@@ -403,7 +393,7 @@ constexpr int P_TMEM_COLS = 2 * P_BN;  // two 256-column accumulators = all 512 
 constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + STG_TOTAL + 1024 + 256;
 
 template <bool B_MN>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
                     const __grid_constant__ CUtensorMap tmDm, const Epilogue epi, int M, int N, int K, int batch,
@@ -431,7 +421,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);   // multicast commit, both CTAs
-      mbar_init(&tempty[a], 8);  // leader's: 4 epilogue warps x 2 CTAs
+      mbar_init(&tempty[a], 2 * EPI_WARPS);  // leader's: every epilogue warp of both CTAs
     }
     *abort = 0;
     fence_mbar_init();
@@ -536,18 +526,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------ epilogue (both CTAs)
-    const int ew = warp - 4;
+    const int ep = warp - 4;
+    const int ew = warp & 3;
+    const int half = ep >> 2;
     int acc = 0;
     uint32_t acc_phase = 0;
     StageState st;
-    uint8_t* wstg = stg + ew * WARP_STG;
+    uint8_t* wstg = stg + ep * WARP_STG;
     for (long long t = pair; t < total; t += npairs) {
       int l, tm, tn;
       bool mir;
       decode_tile(t, per_mat, tiles_m, tiles_n, P_BM, P_BN, sy, l, tm, tn, mir);
-      if (staged)
-        stage_first_c(epi, &tmC, wstg, cbar + ew * NRING, l, tm * P_BM + static_cast<int>(rank) * BM + ew * 32,
-                      tn * P_BN, lane, st);
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, abort));
       if (!ok) break;
       tc_fence_after();
@@ -555,11 +544,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
       const int row = row0 + ew * 32 + lane;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(ew * 32) << 16) + acc * P_BN;
       if (staged) {
-        store_tile_staged<P_BN>(epi, &tmC, &tmD, &tmDm, wstg, cbar + ew * NRING, tbase, l, row0 + ew * 32,
-                                tn * P_BN, M, N, mir, lane, st, abort);
+        store_tile_staged<P_BN>(epi, &tmC, &tmD, &tmDm, wstg, cbar + ep * NRING, tbase, l, row0 + ew * 32,
+                                tn * P_BN, M, N, mir, lane, half, st, abort);
       } else {
 #pragma unroll 1
-        for (int c0 = 0; c0 < P_BN; c0 += 32) {
+        for (int c0 = half * 32; c0 < P_BN; c0 += 32 * (EPI_WARPS / 4)) {
           const int col = tn * P_BN + c0;
           float v[32];
           tmem_ld_32cols(tbase + c0, v);
@@ -653,7 +642,7 @@ cudaError_t launch_one(const TcGemm& g, cudaStream_t s, int* dev_err, int num_sm
   const long long per_mat = tiles_per_matrix(g.M, g.N, BM, BN, g.sym);
   const long long tiles = per_mat * g.batch;
   const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-  tc_gemm_kernel<BN, B_MN><<<grid, 256, C::SMEM_BYTES, s>>>(ma, mb, mc, md, mm, g.epi, g.M, g.N, g.K, g.batch,
+  tc_gemm_kernel<BN, B_MN><<<grid, THREADS, C::SMEM_BYTES, s>>>(ma, mb, mc, md, mm, g.epi, g.M, g.N, g.K, g.batch,
                                                             g.sym ? 1 : 0, per_mat, staged, dev_err);
   return cudaGetLastError();
 }
@@ -669,7 +658,7 @@ cudaError_t launch_pair(const TcGemm& g, cudaStream_t s, int* dev_err, int num_s
     if (attr_err != cudaSuccess) return;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (num_sms / 2));
-    cfg.blockDim = dim3(256);
+    cfg.blockDim = dim3(THREADS);
     cfg.dynamicSmemBytes = P_SMEM_BYTES;
     cudaLaunchAttribute attr;
     attr.id = cudaLaunchAttributeClusterDimension;
@@ -695,7 +684,7 @@ cudaError_t launch_pair(const TcGemm& g, cudaStream_t s, int* dev_err, int num_s
   const long long per_mat = tiles_per_matrix(g.M, g.N, P_BM, P_BN, g.sym);
   const long long tiles = per_mat * g.batch;
   const long long pairs = tiles < max_clusters ? tiles : max_clusters;
-  tc_gemm2_kernel<B_MN><<<static_cast<int>(2 * pairs), 256, P_SMEM_BYTES, s>>>(
+  tc_gemm2_kernel<B_MN><<<static_cast<int>(2 * pairs), THREADS, P_SMEM_BYTES, s>>>(
       ma, mb, mc, md, mm, g.epi, g.M, g.N, g.K, g.batch, g.sym ? 1 : 0, per_mat, staged, dev_err);
   return cudaGetLastError();
 }
