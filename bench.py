@@ -208,7 +208,7 @@ def profile_traffic(kernel_file: Path):
     """Per-launch DRAM traffic of the dominant kernel from the committed ncu
     summary, if it was taken on the current kernel source."""
     import hashlib
-    summ = ROOT / "profiles" / "tc_gemm_batch64-1024x1024.md"
+    summ = ROOT / "profiles" / "tc_gemm_pair_batch64-1024x1024.md"
     if not summ.exists():
         return None
     sha = hashlib.sha256(kernel_file.read_bytes()).hexdigest()[:16]
@@ -230,6 +230,9 @@ def main():
     ap.add_argument("--workload", default="batch64-1024x1024-bf16")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cache-file", default=None,
+                    help="autotune cache: loaded before the warm-up if present, saved after it "
+                         "(lets a profiled run replay the plans of an unprofiled one)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -266,9 +269,13 @@ def main():
             dist.barrier()
 
     # warm-up (first call tunes each shape group and fills the cache)
+    if args.cache_file and os.path.exists(args.cache_file):
+        B.dmuon_cache_load(args.cache_file)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    if args.cache_file and rank == 0:
+        B.dmuon_cache_save(args.cache_file)
     plans = B.dmuon_cache_entries()
 
     clocks = ClockSampler(local)
@@ -347,6 +354,8 @@ def main():
     peak_tc = peaks["bf16_tflops"]
     ach = gemm["flops"] / (gemm["ms"] * 1e-3) / 1e12 if gemm["ms"] > 0 else 0.0
     traffic = profile_traffic(ROOT / "newton_schulz_normalise_b200" / "csrc" / "gemm_tc.cu")
+    tiles = {e.split()[5] for e in plans}
+    gemm_kernel = "tc_gemm2_kernel (CTA pair)" if tiles == {"512"} else "tc_gemm_kernel / tc_gemm2_kernel"
     ew = kinds[B.KIND_EW]
     ew_gbs = ew["bytes"] / (ew["ms"] * 1e-3) / 1e9 if ew["ms"] > 0 else 0.0
 
@@ -364,7 +373,7 @@ def main():
             "ns_tflops": round(tflops, 1),
             "ns_frac_of_peak": round(tflops / peak_tc, 4),
             "ns_tflops_dense_equivalent": round(dense / (ms_per_step * 1e-3) / 1e12, 1),
-            "roofline": {"bound": "tensor", "kernel": "tc_gemm_kernel", "achieved": round(ach, 1),
+            "roofline": {"bound": "tensor", "kernel": gemm_kernel, "achieved": round(ach, 1),
                          "peak": peak_tc, "unit": "TFLOP/s", "frac": round(ach / peak_tc, 4),
                          "traffic": traffic, "peak_source": f"{peaks['_source']} bf16_tflops (burst)",
                          "launches": gemm["launches"] // kt_steps,

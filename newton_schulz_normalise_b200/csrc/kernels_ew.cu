@@ -53,6 +53,14 @@ __device__ __forceinline__ void load8(const void* p, long long i, int is_f32, fl
   }
 }
 
+// Streaming (evict-first) store of 8 fp32 values: the momentum buffer is not
+// read again in this step.
+__device__ __forceinline__ void store8_stream_f32(float* p, long long i, const float (&x)[8]) {
+  float4* q = reinterpret_cast<float4*>(p + i);
+  __stcs(q, make_float4(x[0], x[1], x[2], x[3]));
+  __stcs(q + 1, make_float4(x[4], x[5], x[6], x[7]));
+}
+
 __device__ __forceinline__ void store8(void* p, long long i, int is_f32, const float (&x)[8]) {
   if (is_f32) {
     float4* q = reinterpret_cast<float4*>(static_cast<float*>(p) + i);
@@ -78,10 +86,36 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_wide_kernel(const Momentu
   const float mu = a.mu;
   float ss = 0.f;
   if (vec_ok) {
-    // cols % 8 == 0 and every base 16/32-byte aligned: ldx == cols.
+    // cols % 8 == 0 and every base 16-byte aligned: ldx == cols.  Two
+    // vectors per thread per pass keep twice the bytes in flight.
     const long long nvec = numel / VEC;
-    for (long long v = static_cast<long long>(blockIdx.x) * EW_THREADS + threadIdx.x; v < nvec;
-         v += static_cast<long long>(gridDim.x) * EW_THREADS) {
+    const long long stride = static_cast<long long>(gridDim.x) * EW_THREADS;
+    long long v = static_cast<long long>(blockIdx.x) * EW_THREADS + threadIdx.x;
+    for (; v + stride < nvec; v += 2 * stride) {
+      const long long i0 = v * VEC, i1 = (v + stride) * VEC;
+      float g0[8], b0[8], g1[8], b1[8], u[8];
+      load8(G, i0, a.g_f32, g0);
+      load8(B, i0, 1, b0);
+      load8(G, i1, a.g_f32, g1);
+      load8(B, i1, 1, b1);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        b0[t] = fmaf(mu, b0[t], g0[t]);
+        u[t] = a.nesterov ? fmaf(mu, b0[t], g0[t]) : b0[t];
+        ss = fmaf(u[t], u[t], ss);
+      }
+      store8_stream_f32(B, i0, b0);
+      store8(a.X, xoff + i0, a.x_f32, u);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        b1[t] = fmaf(mu, b1[t], g1[t]);
+        u[t] = a.nesterov ? fmaf(mu, b1[t], g1[t]) : b1[t];
+        ss = fmaf(u[t], u[t], ss);
+      }
+      store8_stream_f32(B, i1, b1);
+      store8(a.X, xoff + i1, a.x_f32, u);
+    }
+    if (v < nvec) {
       const long long i = v * VEC;
       float g[8], b[8], u[8];
       load8(G, i, a.g_f32, g);
@@ -92,7 +126,7 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_wide_kernel(const Momentu
         u[t] = a.nesterov ? fmaf(mu, b[t], g[t]) : b[t];
         ss = fmaf(u[t], u[t], ss);
       }
-      store8(B, i, 1, b);
+      store8_stream_f32(B, i, b);
       store8(a.X, xoff + i, a.x_f32, u);
     }
   } else {
@@ -223,12 +257,12 @@ __global__ void diff_norms_kernel(const void* X, const void* Y, long long ld, in
 
 int momentum_partials(int rows, int cols, int cnt, int num_sms) {
   const long long numel = static_cast<long long>(rows) * cols;
-  long long want = (4LL * num_sms + cnt - 1) / cnt;  // ~4 blocks per SM over the group
+  long long want = (8LL * num_sms + cnt - 1) / cnt;  // ~8 blocks (2048 threads) per SM over the group
   long long cap;
   if (rows > cols)
     cap = static_cast<long long>((rows + TT - 1) / TT) * ((cols + TT - 1) / TT);
   else
-    cap = (numel + EW_THREADS * VEC * 4 - 1) / (EW_THREADS * VEC * 4);  // >= 4 vectors per thread
+    cap = (numel + EW_THREADS * VEC * 2 - 1) / (EW_THREADS * VEC * 2);  // >= 2 vectors per thread
   long long nb = want < cap ? want : cap;
   if (nb < 1) nb = 1;
   if (nb > 4096) nb = 4096;
