@@ -377,7 +377,7 @@ def main():
         line = {
             "metric": METRIC, "value": round(value, 4), "unit": "ms", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
-            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": w.param_dtype,
             "data": "synthetic (seeded N(0,0.02^2) weights, N(0,1e-3^2) grads, zero fp32 momenta)",
             "config": {"workload": w.name, "matrices": len(shapes),
                        "shapes": sorted({f"{r}x{c}" for r, c in shapes}), "ns_steps": w.ns_steps,

@@ -3,36 +3,38 @@
 // The bf16 tensor-core path holds the update to about 1e-2 relative error;
 // fp32 weights are held to 1e-4, which bf16 (or tf32) operands cannot reach.
 // This kernel keeps the whole Newton-Schulz iteration in fp32 FFMA with the
-// same epilogue contract as the tensor-core GEMM.  64x64 output tile per
-// block, 16-deep k slices staged in shared memory, 4x4 outputs per thread.
+// same epilogue contract as the tensor-core GEMM.  32x32 output tile per
+// block of 256 threads (2x2 outputs each), 32-deep k slices staged in shared
+// memory: the fp32 workloads are single matrices of a few hundred rows, so
+// small tiles are what spreads a product over the SMs.
 #include "internal.h"
 
 namespace dmuon {
 
 namespace {
 
-constexpr int TM = 64, TN = 64, TK = 16;
+constexpr int TM = 32, TN = 32, TK = 32;
 
 __global__ void __launch_bounds__(256) simt_gemm_kernel(const float* __restrict__ A, long long lda, long long sa,
                                                         const float* __restrict__ B, long long ldb, long long sb,
                                                         int b_kmajor, int M, int N, int K, const Epilogue epi) {
-  __shared__ float As[TK][TM + 4];
-  __shared__ float Bs[TK][TN + 4];
+  __shared__ float As[TK][TM + 1];
+  __shared__ float Bs[TK][TN + 1];
   const int l = blockIdx.z;
   const int m0 = blockIdx.y * TM, n0 = blockIdx.x * TN;
   const int tid = threadIdx.x;
-  const int tx = tid % 16, ty = tid / 16;
+  const int tx = tid % 16, ty = tid / 16;  // 16 x 16 threads, 2 x 2 outputs each
   const float* Ab = A + static_cast<long long>(l) * sa;
   const float* Bb = B + static_cast<long long>(l) * sb;
-  float acc[4][4] = {};
+  float acc[2][2] = {};
   for (int k0 = 0; k0 < K; k0 += TK) {
-    // A tile: 64 rows x 16 k (k contiguous in memory)
+    // A tile: 32 rows x 32 k (k contiguous in memory): coalesced along k
     for (int i = tid; i < TM * TK; i += 256) {
       const int r = i / TK, k = i % TK;
       const int gr = m0 + r, gk = k0 + k;
       As[k][r] = (gr < M && gk < K) ? Ab[static_cast<long long>(gr) * lda + gk] : 0.f;
     }
-    // B tile: 16 k x 64 cols
+    // B tile: 32 k x 32 columns
     for (int i = tid; i < TN * TK; i += 256) {
       int c, k;
       if (b_kmajor) {
@@ -49,24 +51,21 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const float* __restrict_
       Bs[k][c] = v;
     }
     __syncthreads();
-#pragma unroll
+#pragma unroll 8
     for (int k = 0; k < TK; ++k) {
-      float a[4], b[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = As[k][ty * 4 + i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = Bs[k][tx * 4 + j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+      const float a0 = As[k][ty * 2], a1 = As[k][ty * 2 + 1];
+      const float b0 = Bs[k][tx * 2], b1 = Bs[k][tx * 2 + 1];
+      acc[0][0] = fmaf(a0, b0, acc[0][0]);
+      acc[0][1] = fmaf(a0, b1, acc[0][1]);
+      acc[1][0] = fmaf(a1, b0, acc[1][0]);
+      acc[1][1] = fmaf(a1, b1, acc[1][1]);
     }
     __syncthreads();
   }
-  const int col = n0 + tx * 4;
+  const int col = n0 + tx * 2;
   if (col >= N) return;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) epilogue_row<4>(epi, l, m0 + ty * 4 + i, col, acc[i], M, N);
+  for (int i = 0; i < 2; ++i) epilogue_row<2>(epi, l, m0 + ty * 2 + i, col, acc[i], M, N);
 }
 
 }  // namespace
