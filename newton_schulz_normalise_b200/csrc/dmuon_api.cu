@@ -119,6 +119,11 @@ struct DeviceCtx {
   int* err_host = nullptr;  // mapped pinned word the kernels write on timeout
   int* err_dev = nullptr;
   cudaEvent_t tune_a = nullptr, tune_b = nullptr;
+  // side streams for shape groups too small to fill the GPU on their own
+  static constexpr int kSide = 3;
+  cudaStream_t side[kSide] = {};
+  cudaEvent_t fork_ev = nullptr;
+  cudaEvent_t side_done[kSide] = {};
 };
 
 std::mutex g_ctx_mu;
@@ -144,6 +149,11 @@ int get_ctx(DeviceCtx** out) {
     CUDA_TRY(cudaEventCreateWithFlags(&c->pin_ev[1], cudaEventDisableTiming));
     CUDA_TRY(cudaEventCreate(&c->tune_a));
     CUDA_TRY(cudaEventCreate(&c->tune_b));
+    CUDA_TRY(cudaEventCreateWithFlags(&c->fork_ev, cudaEventDisableTiming));
+    for (int i = 0; i < DeviceCtx::kSide; ++i) {
+      CUDA_TRY(cudaStreamCreateWithFlags(&c->side[i], cudaStreamNonBlocking));
+      CUDA_TRY(cudaEventCreateWithFlags(&c->side_done[i], cudaEventDisableTiming));
+    }
     CUDA_TRY(cudaHostAlloc(reinterpret_cast<void**>(&c->err_host), sizeof(int), cudaHostAllocMapped));
     *c->err_host = 0;
     CUDA_TRY(cudaHostGetDevicePointer(reinterpret_cast<void**>(&c->err_dev), c->err_host, 0));
@@ -706,6 +716,7 @@ int run_step(Request& r) {
   // plans: cache lookup; misses are tuned on this call's data below
   std::vector<Geo> geos(groups.size());
   std::vector<bool> miss(groups.size(), false);
+  std::vector<size_t> needs(groups.size(), 0);
   size_t ws_need = 0;
   for (size_t k = 0; k < groups.size(); ++k) {
     Group& gr = groups[k];
@@ -725,11 +736,55 @@ int run_step(Request& r) {
     Layout L = make_layout(geos[k], gr.chunk, nblk);
     size_t need = L.total;
     if (miss[k]) need += 2 * align256(static_cast<size_t>(gr.chunk) * geos[k].x_elems() * geos[k].esz) + 256;
-    ws_need = std::max(ws_need, need);
+    needs[k] = align256(need);
+  }
+  // Scheduler: groups run in descending measured cost.  Once every plan is
+  // cached, groups whose largest product does not fill the GPU (under two
+  // waves of output tiles) are spread over side streams, longest first onto
+  // the least loaded stream, so they overlap each other and the big groups;
+  // each stream has its own scratch region.
+  const bool any_miss = std::find(miss.begin(), miss.end(), true) != miss.end();
+  std::vector<int> lane(groups.size(), 0);  // 0: the caller's stream; 1..kSide: side streams
+  auto group_cost = [&](int k) {
+    return groups[k].plan.cost_ms * static_cast<double>((groups[k].idx.size() + groups[k].chunk - 1) / groups[k].chunk);
+  };
+  if (!any_miss && !f32 && groups.size() >= 2) {
+    std::vector<int> small;
+    for (size_t k = 0; k < groups.size(); ++k) {
+      const Geo& g = geos[k];
+      const int tl = groups[k].plan.tile;
+      const long long tiles = tc_gemm_tiles(g.m, g.n, groups[k].chunk, tl, false);
+      const long long wave = tl == 512 ? c.num_sms / 2 : c.num_sms;
+      if (groups[k].idx.size() <= static_cast<size_t>(groups[k].chunk) && tiles < 2 * wave)
+        small.push_back(static_cast<int>(k));
+    }
+    std::stable_sort(small.begin(), small.end(), [&](int x, int y) { return group_cost(x) > group_cost(y); });
+    double load[DeviceCtx::kSide] = {0, 0, 0};
+    for (int k : small) {
+      int best = 0;
+      for (int i = 1; i < DeviceCtx::kSide; ++i)
+        if (load[i] < load[best]) best = i;
+      lane[k] = best + 1;
+      load[best] += group_cost(k);
+    }
+  }
+  std::vector<size_t> region_need(DeviceCtx::kSide + 1, 0);
+  std::vector<size_t> region_off(DeviceCtx::kSide + 1, 0);
+  auto layout_regions = [&] {
+    std::fill(region_need.begin(), region_need.end(), 0);
+    for (size_t k = 0; k < groups.size(); ++k) region_need[lane[k]] = std::max(region_need[lane[k]], needs[k]);
+    for (int i = 1; i <= DeviceCtx::kSide; ++i) region_off[i] = region_off[i - 1] + region_need[i - 1];
+    ws_need = region_off[DeviceCtx::kSide] + region_need[DeviceCtx::kSide];
+  };
+  layout_regions();
+  const size_t tables_bytes = align256(4 * sizeof(void*) * static_cast<size_t>(r.count));
+  if (g_ext_ptr && align256(ws_need) + tables_bytes > g_ext_bytes) {
+    std::fill(lane.begin(), lane.end(), 0);  // a caller buffer too small for side streams: one stream
+    layout_regions();
   }
   // device pointer tables: 4 arrays of count pointers, after the chunk scratch
   const size_t tables_off = align256(ws_need);
-  const size_t total_ws = tables_off + align256(4 * sizeof(void*) * static_cast<size_t>(r.count));
+  const size_t total_ws = tables_off + tables_bytes;
   rc = ensure_ws(c, total_ws, r.s);
   if (rc) return rc;
 
@@ -762,20 +817,28 @@ int run_step(Request& r) {
   for (size_t k = 0; k < order.size(); ++k) order[k] = static_cast<int>(k);
   std::stable_sort(order.begin(), order.end(), [&](int x, int y) {
     if (miss[x] != miss[y]) return static_cast<bool>(miss[x]);
-    const double cx = groups[x].plan.cost_ms * ((groups[x].idx.size() + groups[x].chunk - 1) / groups[x].chunk);
-    const double cy = groups[y].plan.cost_ms * ((groups[y].idx.size() + groups[y].chunk - 1) / groups[y].chunk);
-    return cx > cy;
+    return group_cost(x) > group_cost(y);
   });
+  bool side_used[DeviceCtx::kSide] = {false, false, false};
+  for (size_t k = 0; k < groups.size(); ++k)
+    if (lane[k] > 0) side_used[lane[k] - 1] = true;
+  const bool forked = side_used[0] || side_used[1] || side_used[2];
+  if (forked) {
+    CUDA_TRY(cudaEventRecord(c.fork_ev, r.s));
+    for (int i = 0; i < DeviceCtx::kSide; ++i)
+      if (side_used[i]) CUDA_TRY(cudaStreamWaitEvent(c.side[i], c.fork_ev, 0));
+  }
 
   for (int k : order) {
     Group& gr = groups[k];
     const Geo& g = geos[k];
     const int total = static_cast<int>(gr.idx.size());
+    const cudaStream_t gs = lane[k] == 0 ? r.s : c.side[lane[k] - 1];
     for (int c0 = 0; c0 < total; c0 += gr.chunk) {
       Chunk ch;
       ch.g = &g;
       ch.cnt = std::min(gr.chunk, total - c0);
-      ch.base = ws;
+      ch.base = ws + region_off[lane[k]];
       ch.nblk = momentum_partials(g.rows, g.cols, gr.chunk, c.num_sms);
       ch.L = make_layout(g, gr.chunk, ch.nblk);
       const int p = gstart[k] + c0;
@@ -788,11 +851,11 @@ int run_step(Request& r) {
         const int i = gr.idx[c0 + q];
         if (!aligned16(r.grads[i]) || !aligned16(r.moms[i])) ch.aligned = 0;
       }
-      rc = run_momentum(c, ch, f32, g_f32, r.h, r.s);
+      rc = run_momentum(c, ch, f32, g_f32, r.h, gs);
       if (rc) return rc;
       if (miss[k] && c0 == 0) {
         Plan pl;
-        rc = autotune(c, ch, f32, r.h, r.o.variant, &pl, r.s);
+        rc = autotune(c, ch, f32, r.h, r.o.variant, &pl, gs);
         if (rc) return rc;
         gr.plan = pl;
         Key key{gr.rows, gr.cols, f32 ? 1 : 0, r.h.steps, gr.chunk};
@@ -800,12 +863,19 @@ int run_step(Request& r) {
         if (r.o.variant == DMUON_VARIANT_AUTO || !g_cache.count(key)) g_cache[key] = pl;
       }
       Epilogue fin = final_epilogue(r, g, ch, f32);
-      rc = run_ns(c, ch, f32, gr.plan.variant, gr.plan.tile, r.h, fin, ch.cnt, r.s);
+      rc = run_ns(c, ch, f32, gr.plan.variant, gr.plan.tile, r.h, fin, ch.cnt, gs);
       if (rc) return rc;
     }
     if (trace_on())
-      fprintf(stderr, "[dmuon] group %lldx%lld x%d: variant=%d tile=%d chunk=%d cost=%.3f ms\n", gr.rows, gr.cols,
-              total, gr.plan.variant, gr.plan.tile, gr.chunk, gr.plan.cost_ms);
+      fprintf(stderr, "[dmuon] group %lldx%lld x%d: variant=%d tile=%d chunk=%d cost=%.3f ms stream=%d\n", gr.rows,
+              gr.cols, total, gr.plan.variant, gr.plan.tile, gr.chunk, gr.plan.cost_ms, lane[k]);
+  }
+  if (forked) {
+    for (int i = 0; i < DeviceCtx::kSide; ++i)
+      if (side_used[i]) {
+        CUDA_TRY(cudaEventRecord(c.side_done[i], c.side[i]));
+        CUDA_TRY(cudaStreamWaitEvent(r.s, c.side_done[i], 0));
+      }
   }
   CUDA_TRY(cudaEventRecord(c.last_done, r.s));
   c.has_last = true;
@@ -1119,14 +1189,24 @@ int dmuon_workspace_size(const int64_t* shapes, int count, int param_dtype, size
     if (shapes[2 * i] <= 0 || shapes[2 * i + 1] <= 0) return fail(DMUON_ERR_INVALID, "bad shape");
     counts[{shapes[2 * i], shapes[2 * i + 1]}]++;
   }
-  size_t need = 0;
+  // the first call runs every group on one stream (with autotune scratch);
+  // later calls may give up to three small groups a region each
+  size_t need = 0, small_need = 0;
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaGetLastError();
   for (auto& kv : counts) {
     Geo g = make_geo(kv.first.first, kv.first.second, f32);
     int ch = chunk_size(g, kv.second);
-    Layout L = make_layout(g, ch, momentum_partials(g.rows, g.cols, ch, 148));
-    need = std::max(need, L.total + 2 * align256(static_cast<size_t>(ch) * g.x_elems() * g.esz) + 256);
+    Layout L = make_layout(g, ch, momentum_partials(g.rows, g.cols, ch, sms));
+    const size_t n_tune = align256(L.total + 2 * align256(static_cast<size_t>(ch) * g.x_elems() * g.esz) + 256);
+    need = std::max(need, n_tune);
+    const bool maybe_small = !f32 && kv.second <= ch && (tc_gemm_tiles(g.m, g.n, ch, 128, false) < 2LL * sms ||
+                                                         tc_gemm_tiles(g.m, g.n, ch, 512, false) < sms);
+    if (maybe_small) small_need = std::max(small_need, align256(L.total));
   }
-  *bytes = align256(need) + align256(4 * sizeof(void*) * static_cast<size_t>(count));
+  *bytes = need + 3 * small_need + align256(4 * sizeof(void*) * static_cast<size_t>(count));
   return DMUON_OK;
 }
 

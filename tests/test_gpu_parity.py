@@ -141,3 +141,19 @@ def test_gram_and_direct_agree_on_wide(dmuon_lib):
     Og, _ = gpu_update(dmuon_lib, Gs, Ms, variant="gram")
     for i in range(2):
         assert rel_fro(to64(Og[i]), to64(Od[i])) <= 2e-2
+
+
+def test_cached_call_with_side_streams_matches_first_call(dmuon_lib):
+    """The first call on a new set of shapes tunes every group on one stream;
+    later calls run the groups that do not fill the GPU on side streams.
+    Scheduling must not change a single bit of the result."""
+    shapes = [(64, 256)] * 6 + [(256, 1024)] * 3 + [(128, 384)] * 2 + [(1024, 1024)] * 2
+    _, Gs, Ms = make_inputs(shapes, seed=57, m_std=1e-3)
+    O1, B1 = gpu_update(dmuon_lib, Gs, Ms)   # first call: tunes, sequential
+    O2, B2 = gpu_update(dmuon_lib, Gs, Ms)   # cached plans: small groups on side streams
+    O3, B3 = gpu_update(dmuon_lib, Gs, Ms)
+    for i in range(len(shapes)):
+        assert torch.equal(O1[i], O2[i]) and torch.equal(O2[i], O3[i]), i
+        assert torch.equal(B1[i], B2[i])
+        _, Oo = oracle_update(Gs[i], Ms[i])
+        assert rel_fro(to64(O2[i]), Oo) <= BF16_TOL
