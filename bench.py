@@ -329,22 +329,27 @@ def main():
     B.dmuon_timing_reset()
 
     # ---------------- end to end through the C ABI with host buffers
-    # Each step: grads H2D from pinned host memory, the step, params D2H.
+    # dmuon_step_host_io: each step's gradients come from pinned host memory
+    # and the updated parameters go back to pinned host memory; the library
+    # pipelines both copies with the computation, chunk by chunk.
     hG = [g.cpu().pin_memory() for g in Gs]
     hW = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in Ws]
     h2d = sum(x.numel() * x.element_size() for x in hG)
     d2h = sum(x.numel() * x.element_size() for x in hW)
+
+    def step_io():
+        B.dmuon_step_host_io(Ws, hG, Ms, w.lr, w.wd, w.mu, w.ns_steps, params_host_out=hW, opts=opts,
+                             stream=stream)
+
+    for _ in range(2):  # plans of the host-I/O chunking
+        step_io()
     e2e_steps = max(3, min(args.steps, 20))
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        for d, h in zip(Gs, hG):
-            d.copy_(h, non_blocking=True)
-        step()
-        for h, d in zip(hW, Ws):
-            h.copy_(d, non_blocking=True)
+        step_io()
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps

@@ -114,6 +114,29 @@ int dmuon_step_ex(void* const* params, const void* const* grads, void* const* mo
                   int ns_steps, const dmuon_options* opts, void* stream);
 
 /*
+ * dmuon_step_host_io -- dmuon_step_ex for gradients that live in HOST memory
+ * (e.g. reduced or offloaded on the CPU), with the updated parameters copied
+ * back to host memory.  The call splits every shape group into chunks of
+ * about 16 MB of gradients and pipelines them over two internal copy
+ * streams: chunk i+1's gradients travel host->device while chunk i is
+ * computed and chunk i-1's parameters travel device->host, through two
+ * staging slots in the scratch.
+ *   params[i]          device, updated in place (as dmuon_step).
+ *   grads_host[i]      host, rows_i x cols_i row-major; pinned (page-locked)
+ *                      memory for the copies to run asynchronously.
+ *   momenta[i]         device fp32, updated in place.
+ *   params_host_out    NULL (no copy-out) or host pointers that receive the
+ *                      updated parameters (pinned for asynchronous copies).
+ * Asynchronous on `stream`: the host buffers must stay valid, and
+ * params_host_out is complete, only once `stream` has reached the end of the
+ * call's work (e.g. after cudaStreamSynchronize).  Side streams for small
+ * groups are not used in this mode.
+ */
+int dmuon_step_host_io(void* const* params, const void* const* grads_host, void* const* momenta,
+                       void* const* params_host_out, const int64_t* shapes, int count, float lr,
+                       float wd, float mu, int ns_steps, const dmuon_options* opts, void* stream);
+
+/*
  * dmuon_compute_update -- everything but the parameter write: updates the
  * momenta like dmuon_step and writes the orthogonalised update O (before the
  * 0.2*sqrt(max) scale) to out[i], device fp32, rows_i x cols_i row-major.

@@ -32,7 +32,7 @@ EXPORTS = (
     "dmuon_gemm_bf16", "dmuon_cache_save", "dmuon_cache_load", "dmuon_cache_clear",
     "dmuon_cache_size", "dmuon_cache_entry", "dmuon_set_workspace", "dmuon_workspace_size",
     "dmuon_timing_enable", "dmuon_timing_reset", "dmuon_timing_get", "dmuon_launch_count",
-    "dmuon_last_error", "dmuon_version", "dmuon_compute_update_noalloc",
+    "dmuon_last_error", "dmuon_version", "dmuon_compute_update_noalloc", "dmuon_step_host_io",
 )
 
 
@@ -78,6 +78,7 @@ def _load() -> ctypes.CDLL:
         "dmuon_last_error": (ctypes.c_char_p, []),
         "dmuon_version": (I, []),
         "dmuon_compute_update_noalloc": (I, [P, P, I64, I64, F, I, ctypes.POINTER(Options), P, P]),
+        "dmuon_step_host_io": (I, [PP, PP, PP, PP, PI64, I, F, F, F, I, ctypes.POINTER(Options), P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -166,6 +167,22 @@ def dmuon_step_ex(params, grads, momenta, lr, wd, mu, ns_steps=5, opts: Options 
                        _dtype_code(grads[0]) if n else DMUON_BF16, **kw)
     return _check(lib.dmuon_step_ex(_ptrs(params), _ptrs(grads), _ptrs(momenta), _shapes(grads), n,
                                     lr, wd, mu, ns_steps, ctypes.byref(opts), _stream(stream)))
+
+
+def dmuon_step_host_io(params, grads_host, momenta, lr, wd, mu, ns_steps=5, params_host_out=None,
+                       opts: Options | None = None, stream=None, **kw):
+    """Muon step with host-memory gradients (pinned CPU tensors) and an
+    optional host copy of the updated parameters; copies overlap compute."""
+    n = len(params)
+    assert len(grads_host) == n and len(momenta) == n
+    if params_host_out is not None:
+        assert len(params_host_out) == n
+    if opts is None:
+        opts = options(_dtype_code(params[0]) if n else DMUON_BF16,
+                       _dtype_code(grads_host[0]) if n else DMUON_BF16, **kw)
+    out = _ptrs(params_host_out) if params_host_out is not None else None
+    return _check(lib.dmuon_step_host_io(_ptrs(params), _ptrs(grads_host), _ptrs(momenta), out, _shapes(params),
+                                         n, lr, wd, mu, ns_steps, ctypes.byref(opts), _stream(stream)))
 
 
 def dmuon_compute_update(grads, momenta, out, mu, ns_steps=5, opts: Options | None = None, stream=None, **kw):

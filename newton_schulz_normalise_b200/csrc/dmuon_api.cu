@@ -124,6 +124,9 @@ struct DeviceCtx {
   cudaStream_t side[kSide] = {};
   cudaEvent_t fork_ev = nullptr;
   cudaEvent_t side_done[kSide] = {};
+  // host I/O pipeline: copy-in and copy-out streams, two staging slots
+  cudaStream_t cin = nullptr, cout = nullptr;
+  cudaEvent_t g_ready[2] = {}, g_free[2] = {}, w_done[2] = {}, io_done = nullptr;
 };
 
 std::mutex g_ctx_mu;
@@ -154,6 +157,14 @@ int get_ctx(DeviceCtx** out) {
       CUDA_TRY(cudaStreamCreateWithFlags(&c->side[i], cudaStreamNonBlocking));
       CUDA_TRY(cudaEventCreateWithFlags(&c->side_done[i], cudaEventDisableTiming));
     }
+    CUDA_TRY(cudaStreamCreateWithFlags(&c->cin, cudaStreamNonBlocking));
+    CUDA_TRY(cudaStreamCreateWithFlags(&c->cout, cudaStreamNonBlocking));
+    for (int i = 0; i < 2; ++i) {
+      CUDA_TRY(cudaEventCreateWithFlags(&c->g_ready[i], cudaEventDisableTiming));
+      CUDA_TRY(cudaEventCreateWithFlags(&c->g_free[i], cudaEventDisableTiming));
+      CUDA_TRY(cudaEventCreateWithFlags(&c->w_done[i], cudaEventDisableTiming));
+    }
+    CUDA_TRY(cudaEventCreateWithFlags(&c->io_done, cudaEventDisableTiming));
     CUDA_TRY(cudaHostAlloc(reinterpret_cast<void**>(&c->err_host), sizeof(int), cudaHostAllocMapped));
     *c->err_host = 0;
     CUDA_TRY(cudaHostGetDevicePointer(reinterpret_cast<void**>(&c->err_dev), c->err_host, 0));
@@ -512,6 +523,8 @@ struct Request {
   Hyper h;
   dmuon_options o;
   cudaStream_t s;
+  bool grads_host = false;             // dmuon_step_host_io: grads in host memory
+  void* const* params_host = nullptr;  // dmuon_step_host_io: updated params copied here
 };
 
 int validate(const Request& r) {
@@ -535,7 +548,8 @@ int validate(const Request& r) {
     if (rr <= 0 || cc <= 0) return fail(DMUON_ERR_INVALID, "matrix %d has shape %lld x %lld", i, (long long)rr, (long long)cc);
     if (rr > (1 << 20) || cc > (1 << 20) || rr * cc > (1LL << 31))
       return fail(DMUON_ERR_INVALID, "matrix %d shape %lld x %lld too large", i, (long long)rr, (long long)cc);
-    if (!r.grads[i] || !r.moms[i] || (r.params && !r.params[i]) || (r.out && !r.out[i]))
+    if (!r.grads[i] || !r.moms[i] || (r.params && !r.params[i]) || (r.out && !r.out[i]) ||
+        (r.params_host && !r.params_host[i]))
       return fail(DMUON_ERR_INVALID, "null pointer for matrix %d", i);
   }
   return DMUON_OK;
@@ -684,6 +698,17 @@ int autotune(DeviceCtx& c, const Chunk& ch, bool f32, const Hyper& h, int forced
 }
 
 
+// Host I/O pipeline: matrices per chunk (about 16 MB of gradients, at least
+// one matrix) and the 256-byte aligned stride of one staged gradient.
+int io_chunk(long long rows, long long cols, bool g_f32) {
+  const long long bytes = rows * cols * (g_f32 ? 4 : 2);
+  const long long n = (16LL << 20) / std::max(bytes, 1LL);
+  return static_cast<int>(std::max(1LL, std::min(n, 65535LL)));
+}
+size_t io_stride(long long rows, long long cols, bool g_f32) {
+  return align256(static_cast<size_t>(rows * cols * (g_f32 ? 4 : 2)));
+}
+
 int run_step(Request& r) {
   int rc = validate(r);
   if (rc || r.count == 0) return rc;
@@ -718,10 +743,12 @@ int run_step(Request& r) {
   std::vector<bool> miss(groups.size(), false);
   std::vector<size_t> needs(groups.size(), 0);
   size_t ws_need = 0;
+  size_t stage_slot = 0;  // host I/O: bytes of one staging slot for gradients
   for (size_t k = 0; k < groups.size(); ++k) {
     Group& gr = groups[k];
     geos[k] = make_geo(gr.rows, gr.cols, f32);
     gr.chunk = chunk_size(geos[k], static_cast<int>(gr.idx.size()));
+    if (r.grads_host) gr.chunk = std::min(gr.chunk, io_chunk(gr.rows, gr.cols, g_f32));
     Key key{gr.rows, gr.cols, f32 ? 1 : 0, r.h.steps, gr.chunk};
     {
       std::lock_guard<std::mutex> lk2(g_cache_mu);
@@ -737,6 +764,7 @@ int run_step(Request& r) {
     size_t need = L.total;
     if (miss[k]) need += 2 * align256(static_cast<size_t>(gr.chunk) * geos[k].x_elems() * geos[k].esz) + 256;
     needs[k] = align256(need);
+    if (r.grads_host) stage_slot = std::max(stage_slot, static_cast<size_t>(gr.chunk) * io_stride(gr.rows, gr.cols, g_f32));
   }
   // Scheduler: groups run in descending measured cost.  Once every plan is
   // cached, groups whose largest product does not fill the GPU (under two
@@ -748,7 +776,7 @@ int run_step(Request& r) {
   auto group_cost = [&](int k) {
     return groups[k].plan.cost_ms * static_cast<double>((groups[k].idx.size() + groups[k].chunk - 1) / groups[k].chunk);
   };
-  if (!any_miss && !f32 && groups.size() >= 2) {
+  if (!any_miss && !f32 && groups.size() >= 2 && !r.grads_host) {
     std::vector<int> small;
     for (size_t k = 0; k < groups.size(); ++k) {
       const Geo& g = geos[k];
@@ -783,7 +811,8 @@ int run_step(Request& r) {
     layout_regions();
   }
   // device pointer tables: 4 arrays of count pointers, after the chunk scratch
-  const size_t tables_off = align256(ws_need);
+  const size_t stage_off = align256(ws_need);  // host I/O: two gradient staging slots
+  const size_t tables_off = stage_off + 2 * align256(stage_slot);
   const size_t total_ws = tables_off + tables_bytes;
   rc = ensure_ws(c, total_ws, r.s);
   if (rc) return rc;
@@ -791,7 +820,18 @@ int run_step(Request& r) {
   // order GPU work after the previous call's (it may be on another stream)
   if (c.has_last) CUDA_TRY(cudaStreamWaitEvent(r.s, c.last_done, 0));
 
-  // pointer tables, grouped: for group k, its matrices are contiguous
+  // issue order: tuned groups first (they synchronise), then by cost
+  std::vector<int> order(groups.size());
+  for (size_t k = 0; k < order.size(); ++k) order[k] = static_cast<int>(k);
+  std::stable_sort(order.begin(), order.end(), [&](int x, int y) {
+    if (miss[x] != miss[y]) return static_cast<bool>(miss[x]);
+    return group_cost(x) > group_cost(y);
+  });
+
+  // pointer tables, grouped: for group k, its matrices are contiguous.  With
+  // host gradients the G entries point at the staging slot of the matrix's
+  // chunk (chunks alternate between the two slots in issue order).
+  uint8_t* ws = static_cast<uint8_t*>(c.ws);
   std::vector<void*> host(4 * static_cast<size_t>(r.count));
   std::vector<int> gstart(groups.size());
   {
@@ -806,19 +846,27 @@ int run_step(Request& r) {
         ++pos;
       }
     }
+    if (r.grads_host) {
+      int j = 0;
+      for (int k : order) {
+        const Group& gr = groups[k];
+        const size_t stride = io_stride(gr.rows, gr.cols, g_f32);
+        const int total = static_cast<int>(gr.idx.size());
+        for (int c0 = 0; c0 < total; c0 += gr.chunk, ++j)
+          for (int q = 0; q < std::min(gr.chunk, total - c0); ++q)
+            host[gstart[k] + c0 + q] = ws + stage_off + (j & 1) * align256(stage_slot) + q * stride;
+      }
+    }
   }
-  uint8_t* ws = static_cast<uint8_t*>(c.ws);
   void** dtab = reinterpret_cast<void**>(ws + tables_off);
   rc = upload_tables(c, host, dtab, r.s);
   if (rc) return rc;
-
-  // issue order: tuned groups first (they synchronise), then by cost
-  std::vector<int> order(groups.size());
-  for (size_t k = 0; k < order.size(); ++k) order[k] = static_cast<int>(k);
-  std::stable_sort(order.begin(), order.end(), [&](int x, int y) {
-    if (miss[x] != miss[y]) return static_cast<bool>(miss[x]);
-    return group_cost(x) > group_cost(y);
-  });
+  if (r.grads_host) {  // the copy streams start after everything before this call
+    CUDA_TRY(cudaEventRecord(c.fork_ev, r.s));
+    CUDA_TRY(cudaStreamWaitEvent(c.cin, c.fork_ev, 0));
+    CUDA_TRY(cudaStreamWaitEvent(c.cout, c.fork_ev, 0));
+  }
+  int io_j = 0;  // host I/O: chunk counter in issue order
   bool side_used[DeviceCtx::kSide] = {false, false, false};
   for (size_t k = 0; k < groups.size(); ++k)
     if (lane[k] > 0) side_used[lane[k] - 1] = true;
@@ -851,8 +899,20 @@ int run_step(Request& r) {
         const int i = gr.idx[c0 + q];
         if (!aligned16(r.grads[i]) || !aligned16(r.moms[i])) ch.aligned = 0;
       }
+      const int slot = io_j & 1;
+      if (r.grads_host) {
+        // copy-in: this chunk's gradients into its staging slot, once the
+        // chunk two back has consumed that slot
+        if (io_j >= 2) CUDA_TRY(cudaStreamWaitEvent(c.cin, c.g_free[slot], 0));
+        const size_t bytes = static_cast<size_t>(g.rows) * g.cols * (g_f32 ? 4 : 2);
+        for (int q = 0; q < ch.cnt; ++q)
+          CUDA_TRY(cudaMemcpyAsync(host[p + q], r.grads[gr.idx[c0 + q]], bytes, cudaMemcpyHostToDevice, c.cin));
+        CUDA_TRY(cudaEventRecord(c.g_ready[slot], c.cin));
+        CUDA_TRY(cudaStreamWaitEvent(gs, c.g_ready[slot], 0));
+      }
       rc = run_momentum(c, ch, f32, g_f32, r.h, gs);
       if (rc) return rc;
+      if (r.grads_host) CUDA_TRY(cudaEventRecord(c.g_free[slot], gs));
       if (miss[k] && c0 == 0) {
         Plan pl;
         rc = autotune(c, ch, f32, r.h, r.o.variant, &pl, gs);
@@ -865,6 +925,18 @@ int run_step(Request& r) {
       Epilogue fin = final_epilogue(r, g, ch, f32);
       rc = run_ns(c, ch, f32, gr.plan.variant, gr.plan.tile, r.h, fin, ch.cnt, gs);
       if (rc) return rc;
+      if (r.grads_host) {
+        if (r.params_host) {  // copy-out: the chunk's updated parameters
+          CUDA_TRY(cudaEventRecord(c.w_done[slot], gs));
+          CUDA_TRY(cudaStreamWaitEvent(c.cout, c.w_done[slot], 0));
+          const size_t bytes = static_cast<size_t>(g.rows) * g.cols * (f32 ? 4 : 2);
+          for (int q = 0; q < ch.cnt; ++q) {
+            const int i = gr.idx[c0 + q];
+            CUDA_TRY(cudaMemcpyAsync(r.params_host[i], r.params[i], bytes, cudaMemcpyDeviceToHost, c.cout));
+          }
+        }
+        ++io_j;
+      }
     }
     if (trace_on())
       fprintf(stderr, "[dmuon] group %lldx%lld x%d: variant=%d tile=%d chunk=%d cost=%.3f ms stream=%d\n", gr.rows,
@@ -876,6 +948,12 @@ int run_step(Request& r) {
         CUDA_TRY(cudaEventRecord(c.side_done[i], c.side[i]));
         CUDA_TRY(cudaStreamWaitEvent(r.s, c.side_done[i], 0));
       }
+  }
+  if (r.grads_host) {  // join the copy streams back into the caller's stream
+    CUDA_TRY(cudaEventRecord(c.io_done, c.cout));
+    CUDA_TRY(cudaStreamWaitEvent(r.s, c.io_done, 0));
+    CUDA_TRY(cudaEventRecord(c.io_done, c.cin));
+    CUDA_TRY(cudaStreamWaitEvent(r.s, c.io_done, 0));
   }
   CUDA_TRY(cudaEventRecord(c.last_done, r.s));
   c.has_last = true;
@@ -967,6 +1045,21 @@ int dmuon_step_ex(void* const* params, const void* const* grads, void* const* mo
 int dmuon_step(void* const* params, const void* const* grads, void* const* momenta, const int64_t* shapes, int count,
                float lr, float wd, float mu, int ns_steps, void* stream) {
   return dmuon_step_ex(params, grads, momenta, shapes, count, lr, wd, mu, ns_steps, nullptr, stream);
+}
+
+int dmuon_step_host_io(void* const* params, const void* const* grads_host, void* const* momenta,
+                       void* const* params_host_out, const int64_t* shapes, int count, float lr, float wd, float mu,
+                       int ns_steps, const dmuon_options* opts, void* stream) {
+  t_err.clear();
+  dmuon_options o;
+  dmuon_options_init(&o);
+  if (opts) o = *opts;
+  if (!params && count > 0) return fail(DMUON_ERR_INVALID, "params is NULL");
+  Request r{params, grads_host, momenta, nullptr, shapes, count, hyper_from(lr, wd, mu, ns_steps, o), o,
+            static_cast<cudaStream_t>(stream)};
+  r.grads_host = true;
+  r.params_host = params_host_out;
+  return run_step(r);
 }
 
 int dmuon_compute_update(const void* const* grads, void* const* momenta, const int64_t* shapes, int count, float mu,
