@@ -71,7 +71,9 @@ typedef enum dmuon_variant {
   DMUON_VARIANT_AUTO = 0,
   DMUON_VARIANT_DIRECT = 1,  /* iterate on X (m x n): 5 x (m^2 n + m^3 + m^2 n) GEMMs */
   DMUON_VARIANT_GRAM = 2,    /* iterate on Q (m x m), one m x m x n product at the end */
-  DMUON_VARIANT_BATCHED = 3  /* one CTA per small matrix, everything resident on chip */
+  DMUON_VARIANT_BATCHED = 3  /* resident: up to 8 small matrices (m <= 128, n <= 512, bf16) per CTA,
+                                iterate, A and P in shared memory for all steps; other shapes
+                                run as AUTO */
 } dmuon_variant;
 
 /* Options of dmuon_step_ex.  Zero-initialise, then call dmuon_options_init. */

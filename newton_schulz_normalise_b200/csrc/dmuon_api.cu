@@ -418,6 +418,16 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
     if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "scale epilogue: %s", cudaGetErrorString(e));
     return DMUON_OK;
   }
+  if (variant == DMUON_VARIANT_BATCHED) {  // resident small-matrix kernel (bf16 only)
+    cudaError_t e = launch_k(KIND_TC_GEMM, 2.0 * h.steps * (2.0 * 128 * 128 * g.n + 2.0 * 128 * 128 * 128) *
+                                               ((cnt + ns_small_group(m) - 1) / ns_small_group(m)),
+                             0.0, s, [&] {
+                               return launch_ns_small(X0, g.ldx, sv, s2v, cnt, m, n, h.steps, h.a, h.b, h.c, fin, s,
+                                                      c.err_dev);
+                             });
+    if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "resident small-matrix kernel: %s", cudaGetErrorString(e));
+    return DMUON_OK;
+  }
   if (variant == DMUON_VARIANT_GRAM) {
     // Every m x m product takes its right operand as stored (MN-major B), not
     // as the transpose of a matrix that is symmetric only up to rounding:
@@ -642,12 +652,19 @@ int autotune(DeviceCtx& c, const Chunk& ch, bool f32, const Hyper& h, int forced
   std::vector<int> vars;
   if (forced_variant == DMUON_VARIANT_DIRECT || forced_variant == DMUON_VARIANT_GRAM)
     vars = {forced_variant};
+  else if (forced_variant == DMUON_VARIANT_BATCHED)
+    vars = {DMUON_VARIANT_DIRECT};  // reference for the gate; the batched candidate is added below
   else {
     vars = {DMUON_VARIANT_DIRECT};
     if (g.n * 4 >= g.m * 5 && h.steps > 0) vars.push_back(DMUON_VARIANT_GRAM);  // n >= 1.25 m
   }
   for (int v : vars)
     for (int t : tiles) cands.push_back({v, t});
+  if (!f32 && ns_small_supported(g.m, g.n) &&
+      (forced_variant == DMUON_VARIANT_AUTO || forced_variant == DMUON_VARIANT_BATCHED))
+    cands.push_back({DMUON_VARIANT_BATCHED, 128});
+  if (forced_variant == DMUON_VARIANT_BATCHED && !cands.empty() && cands.back().first == DMUON_VARIANT_BATCHED)
+    cands = {{DMUON_VARIANT_DIRECT, tiles[0]}, cands.back()};  // direct stays the gate's reference
   if (h.steps == 0) cands = {{DMUON_VARIANT_DIRECT, tiles[0]}};
 
   const int probe = ch.cnt;
@@ -660,6 +677,8 @@ int autotune(DeviceCtx& c, const Chunk& ch, bool f32, const Hyper& h, int forced
   float best = 1e30f;
   Plan bestp;
   bool have_ref = false;
+  bool forced_batched_ok = false;
+  double forced_batched_ms = 0.0;
   for (auto [v, tile] : cands) {
     const bool is_ref = !have_ref;
     void* dst = is_ref ? ref_out : cand_out;
@@ -686,12 +705,21 @@ int autotune(DeviceCtx& c, const Chunk& ch, bool f32, const Hyper& h, int forced
       fprintf(stderr, "[dmuon] tune %dx%d cnt=%d variant=%d tile=%d: %.3f ms%s gate=%.2e %s\n", g.rows, g.cols, probe,
               v, tile, ms, is_ref ? " (reference)" : "", relerr, pass ? "pass" : "REJECT");
     have_ref = true;
+    if (v == DMUON_VARIANT_BATCHED && pass) {
+      forced_batched_ok = true;
+      forced_batched_ms = ms;
+    }
     if (pass && ms < best) {
       best = ms;
       bestp.variant = v;
       bestp.tile = tile;
       bestp.cost_ms = ms;
     }
+  }
+  if (forced_variant == DMUON_VARIANT_BATCHED && forced_batched_ok) {
+    bestp.variant = DMUON_VARIANT_BATCHED;
+    bestp.tile = 128;
+    bestp.cost_ms = forced_batched_ms;
   }
   *plan = bestp;
   return DMUON_OK;
@@ -753,7 +781,11 @@ int run_step(Request& r) {
     {
       std::lock_guard<std::mutex> lk2(g_cache_mu);
       auto it = g_cache.find(key);
-      if (it != g_cache.end() && (r.o.variant == DMUON_VARIANT_AUTO || it->second.variant == r.o.variant)) {
+      // a forced variant the shape cannot take (the resident kernel needs
+      // bf16, m <= 128, n <= 512) runs as planned for AUTO
+      const bool forced_ok = r.o.variant != DMUON_VARIANT_BATCHED || (!f32 && ns_small_supported(geos[k].m, geos[k].n));
+      const int want = forced_ok ? r.o.variant : DMUON_VARIANT_AUTO;
+      if (it != g_cache.end() && (want == DMUON_VARIANT_AUTO || it->second.variant == want)) {
         gr.plan = it->second;
       } else {
         miss[k] = true;
@@ -1226,7 +1258,7 @@ int dmuon_cache_load(const char* path) {
   int f32, steps, cnt, var, tile;
   double cost;
   while (fscanf(f, "%lld %lld %d %d %d %d %d %lf", &rr, &cc, &f32, &steps, &cnt, &var, &tile, &cost) == 8) {
-    if (rr <= 0 || cc <= 0 || cnt <= 0 || (var != 1 && var != 2) || (tile != 128 && tile != 256 && tile != 512)) {
+    if (rr <= 0 || cc <= 0 || cnt <= 0 || var < 1 || var > 3 || (tile != 128 && tile != 256 && tile != 512)) {
       fclose(f);
       return fail(DMUON_ERR_INVALID, "%s: malformed entry", path);
     }
@@ -1259,7 +1291,8 @@ int dmuon_cache_entry(int i, char* buf, size_t len) {
   auto it = g_cache.begin();
   std::advance(it, i);
   snprintf(buf, len, "%lld %lld %s %d %s %d %d %.4f", it->first.rows, it->first.cols, it->first.f32 ? "f32" : "bf16",
-           it->first.steps, it->second.variant == DMUON_VARIANT_GRAM ? "gram" : "direct", it->second.tile, it->first.cnt,
+           it->first.steps, it->second.variant == DMUON_VARIANT_GRAM ? "gram" : (it->second.variant == DMUON_VARIANT_BATCHED ? "batched" : "direct"),
+           it->second.tile, it->first.cnt,
            it->second.cost_ms);
   return DMUON_OK;
 }

@@ -71,6 +71,13 @@ cudaError_t launch_norm_finalize(const float* partials, int nblk, int cnt, float
 cudaError_t launch_scale_epilogue(const void* X, long long ldx, int x_f32, int m, int n, int cnt,
                                   const float* s, const Epilogue& epi, cudaStream_t st);
 
+// Resident Newton-Schulz for small matrices (m <= 128, n <= 512), direct form,
+// one CTA per block of up to 8 stacked matrices; ends with `fin`.
+bool ns_small_supported(int m, int n);
+int ns_small_group(int m);
+cudaError_t launch_ns_small(const void* X0, long long ldx, const float* s, const float* s2, int cnt, int m, int n,
+                            int steps, float a, float b, float c, const Epilogue& fin, cudaStream_t st, int* err);
+
 // Relative Frobenius distance helper for the autotuner's accuracy gate:
 // acc[0] += sum (x - y)^2, acc[1] += sum y^2 over cnt matrices m x n (ld).
 cudaError_t launch_diff_norms(const void* X, const void* Y, long long ld, int m, int n, int cnt, int is_f32,

@@ -38,7 +38,7 @@ def _wide_enough(shapes):
     return all(max(r, c) >= 1.9 * min(r, c) for r, c in shapes)
 
 
-CASES = [(s, v) for s in SMALL_SHAPES for v in ("direct", "gram", "auto")
+CASES = [(s, v) for s in SMALL_SHAPES for v in ("direct", "gram", "auto", "batched")
          if v != "gram" or _wide_enough(s)]
 
 
@@ -76,7 +76,7 @@ def test_fp32_single_256x512_matches_oracle(dmuon_lib):
 def test_ns_steps(dmuon_lib, steps):
     shapes = [(96, 200), (200, 96)]
     Ws, Gs, Ms = make_inputs(shapes, seed=23)
-    for variant in ("direct", "gram"):
+    for variant in ("direct", "gram", "batched"):
         Os, _ = gpu_update(dmuon_lib, Gs, Ms, steps=steps, variant=variant)
         for i in range(2):
             _, Oo = oracle_update(Gs[i], Ms[i], steps=steps)
@@ -157,3 +157,25 @@ def test_cached_call_with_side_streams_matches_first_call(dmuon_lib):
         assert torch.equal(B1[i], B2[i])
         _, Oo = oracle_update(Gs[i], Ms[i])
         assert rel_fro(to64(O2[i]), Oo) <= BF16_TOL
+
+
+@pytest.mark.parametrize("shapes", [[(64, 256)] * 5, [(17, 33)] * 9, [(128, 512)] * 3, [(300, 100)] * 2,
+                                    [(1, 64)] * 11, [(8, 8)] * 3, [(120, 500)]],
+                         ids=["64x256x5", "17x33x9", "128x512x3", "300x100x2", "1x64x11", "8x8x3", "120x500"])
+def test_resident_small_kernel(dmuon_lib, shapes):
+    """The resident kernel (up to 8 matrices stacked per CTA, all steps on
+    chip) against the oracle, and against the direct form it restates."""
+    Ws, Gs, Ms = make_inputs(shapes, seed=91, m_std=1e-3)
+    Ob, Bb = gpu_update(dmuon_lib, Gs, Ms, variant="batched")
+    Od, _ = gpu_update(dmuon_lib, Gs, Ms, variant="direct")
+    for i in range(len(shapes)):
+        _, Oo = oracle_update(Gs[i], Ms[i])
+        assert rel_fro(to64(Ob[i]), Oo) <= BF16_TOL, i
+        assert rel_fro(to64(Ob[i]), to64(Od[i])) <= 1e-2, i
+        check_momentum(Bb[i], Gs[i], Ms[i], 0.95)
+    # and the fused parameter write
+    Wg, _ = gpu_step(dmuon_lib, Ws, Gs, Ms, variant="batched")
+    for i, (r, c) in enumerate(shapes):
+        w_apply = ora.apply_update(to64(Ws[i]), to64(Ob[i]), 0.02, 0.1)
+        terms = np.abs(0.998 * to64(Ws[i])) + np.abs(0.02 * ora.rms_scale(r, c) * to64(Ob[i]))
+        assert np.all(np.abs(to64(Wg[i]) - w_apply) <= np.abs(w_apply) * 2.0 ** -8 + terms * 1e-6), i
