@@ -228,6 +228,16 @@ void dmuon_timing_enable(int enable);
 void dmuon_timing_reset(void);
 int dmuon_timing_get(int kind, int64_t* launches, double* ms, double* flops, double* bytes);
 
+/*
+ * dmuon_selftest_wait -- checks the device-side failure path: launches a
+ * one-block kernel whose mbarrier wait nothing completes, with a limit of
+ * limit_ms (1..2000).  The kernel gives up, records the timeout in the
+ * host-visible error word and returns; the call synchronises `stream` and
+ * returns DMUON_ERR_DEVICE_TIMEOUT when that path works (DMUON_OK would mean
+ * the wait did not time out).  The context stays usable afterwards.
+ */
+int dmuon_selftest_wait(int limit_ms, void* stream);
+
 /* Number of kernels the library launched since load (all kinds). */
 int64_t dmuon_launch_count(void);
 

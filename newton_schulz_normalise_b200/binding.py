@@ -33,6 +33,7 @@ EXPORTS = (
     "dmuon_cache_size", "dmuon_cache_entry", "dmuon_set_workspace", "dmuon_workspace_size",
     "dmuon_timing_enable", "dmuon_timing_reset", "dmuon_timing_get", "dmuon_launch_count",
     "dmuon_last_error", "dmuon_version", "dmuon_compute_update_noalloc", "dmuon_step_host_io",
+    "dmuon_selftest_wait",
 )
 
 
@@ -79,6 +80,7 @@ def _load() -> ctypes.CDLL:
         "dmuon_version": (I, []),
         "dmuon_compute_update_noalloc": (I, [P, P, I64, I64, F, I, ctypes.POINTER(Options), P, P]),
         "dmuon_step_host_io": (I, [PP, PP, PP, PP, PI64, I, F, F, F, I, ctypes.POINTER(Options), P]),
+        "dmuon_selftest_wait": (I, [I, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -281,6 +283,12 @@ def dmuon_timing_get(kind: int):
     ms, fl, by = ctypes.c_double(0), ctypes.c_double(0), ctypes.c_double(0)
     _check(lib.dmuon_timing_get(kind, ctypes.byref(n), ctypes.byref(ms), ctypes.byref(fl), ctypes.byref(by)))
     return {"launches": n.value, "ms": ms.value, "flops": fl.value, "bytes": by.value}
+
+
+def dmuon_selftest_wait(limit_ms: int = 50, stream=None) -> int:
+    """Runs the bounded-wait self-test; returns the raw status (DMUON_ERR_DEVICE_TIMEOUT
+    when the device-side timeout path works)."""
+    return lib.dmuon_selftest_wait(limit_ms, _stream(stream))
 
 
 def dmuon_launch_count() -> int:

@@ -1212,6 +1212,25 @@ int dmuon_gemm_bf16(const void* A, int64_t lda, int64_t sa, const void* B, int64
   return DMUON_OK;
 }
 
+int dmuon_selftest_wait(int limit_ms, void* stream) {
+  t_err.clear();
+  if (limit_ms < 1 || limit_ms > 2000) return fail(DMUON_ERR_INVALID, "limit_ms must be in [1, 2000]");
+  DeviceCtx* cp = nullptr;
+  int rc = get_ctx(&cp);
+  if (rc) return rc;
+  std::lock_guard<std::mutex> lk(cp->mu);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  *cp->err_host = 0;
+  cudaError_t e = launch_wait_selftest(cp->err_dev, static_cast<unsigned long long>(limit_ms) * 1000000ull, s);
+  if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "self-test launch: %s", cudaGetErrorString(e));
+  CUDA_TRY(cudaStreamSynchronize(s));
+  const int word = *cp->err_host;
+  *cp->err_host = 0;  // reported here: the next call starts clean
+  if (word == DMUON_ERR_DEVICE_TIMEOUT)
+    return fail(DMUON_ERR_DEVICE_TIMEOUT, "device wait gave up after %d ms (expected by the self-test)", limit_ms);
+  return DMUON_OK;
+}
+
 int dmuon_cache_save(const char* path) {
   t_err.clear();
   if (!path) return fail(DMUON_ERR_INVALID, "null path");

@@ -78,6 +78,10 @@ int ns_small_group(int m);
 cudaError_t launch_ns_small(const void* X0, long long ldx, const float* s, const float* s2, int cnt, int m, int n,
                             int steps, float a, float b, float c, const Epilogue& fin, cudaStream_t st, int* err);
 
+// One-block kernel whose only mbarrier wait can never complete; it gives up
+// after limit_ns and records kErrTimeout in *err.
+cudaError_t launch_wait_selftest(int* err, unsigned long long limit_ns, cudaStream_t st);
+
 // Relative Frobenius distance helper for the autotuner's accuracy gate:
 // acc[0] += sum (x - y)^2, acc[1] += sum y^2 over cnt matrices m x n (ld).
 cudaError_t launch_diff_norms(const void* X, const void* Y, long long ld, int m, int n, int cnt, int is_f32,

@@ -253,7 +253,27 @@ __global__ void diff_norms_kernel(const void* X, const void* Y, long long ld, in
   }
 }
 
+// Waits on an mbarrier that nothing arrives on, with a short limit: the
+// bounded-wait machinery of the GEMM kernels, exercised on its own.
+__global__ void wait_selftest_kernel(int* err, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait_limit(&bar, 0, &abort, limit_ns) && err)
+    *reinterpret_cast<volatile int*>(err) = kErrTimeout;
+}
+
 }  // namespace
+
+cudaError_t launch_wait_selftest(int* err, unsigned long long limit_ns, cudaStream_t st) {
+  wait_selftest_kernel<<<1, 32, 0, st>>>(err, limit_ns);
+  return cudaGetLastError();
+}
 
 int momentum_partials(int rows, int cols, int cnt, int num_sms) {
   const long long numel = static_cast<long long>(rows) * cols;
