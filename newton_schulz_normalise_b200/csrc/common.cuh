@@ -78,6 +78,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   return mbar_wait_limit(bar, parity, abort, kWaitLimitNs);
 }
 
+// ---------------------------------------------------------------- dependent launch
+// With programmatic dependent launch a kernel may start before the previous
+// kernel on the stream has finished: everything before grid_dep_wait() must
+// not touch memory that kernel writes or reads.  grid_dep_launch() lets the
+// next kernel start its own prologue.  Both are no-ops without the launch
+// attribute.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");

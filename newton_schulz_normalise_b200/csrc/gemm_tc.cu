@@ -249,6 +249,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  grid_dep_wait();  // the previous kernel's results are complete and visible from here on
 
   const int tiles_m = (M + BM - 1) / BM;
   const int tiles_n = (N + BN - 1) / BN;
@@ -374,6 +375,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 
   if (warp >= 4 && lane == 0) bulk_wait<0>();  // each warp's staged stores complete before the CTA exits
+  grid_dep_launch();
   __syncthreads();
   if (*abort && threadIdx.x == 0 && err) *reinterpret_cast<volatile int*>(err) = kErrTimeout;
   if (warp == 2) {
@@ -439,6 +441,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   cluster_sync();  // both CTAs' barriers initialised before any cross-CTA signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  grid_dep_wait();  // the previous kernel's results are complete and visible from here on
 
   const int tiles_m = (M + P_BM - 1) / P_BM;
   const int tiles_n = (N + P_BN - 1) / P_BN;
@@ -566,6 +569,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   }
 
   if (warp >= 4 && lane == 0) bulk_wait<0>();  // each warp's staged stores complete before the CTA exits
+  grid_dep_launch();
   __syncthreads();
   cluster_sync();  // no CTA leaves while its peer may still signal its barriers
   if (*abort && threadIdx.x == 0 && err) *reinterpret_cast<volatile int*>(err) = kErrTimeout;
@@ -642,9 +646,18 @@ cudaError_t launch_one(const TcGemm& g, cudaStream_t s, int* dev_err, int num_sm
   const long long per_mat = tiles_per_matrix(g.M, g.N, BM, BN, g.sym);
   const long long tiles = per_mat * g.batch;
   const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-  tc_gemm_kernel<BN, B_MN><<<grid, THREADS, C::SMEM_BYTES, s>>>(ma, mb, mc, md, mm, g.epi, g.M, g.N, g.K, g.batch,
-                                                            g.sym ? 1 : 0, per_mat, staged, dev_err);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc_gemm_kernel<BN, B_MN>, ma, mb, mc, md, mm, g.epi, g.M, g.N, g.K, g.batch,
+                            g.sym ? 1 : 0, per_mat, staged, dev_err);
 }
 
 template <bool B_MN>
@@ -684,9 +697,18 @@ cudaError_t launch_pair(const TcGemm& g, cudaStream_t s, int* dev_err, int num_s
   const long long per_mat = tiles_per_matrix(g.M, g.N, P_BM, P_BN, g.sym);
   const long long tiles = per_mat * g.batch;
   const long long pairs = tiles < max_clusters ? tiles : max_clusters;
-  tc_gemm2_kernel<B_MN><<<static_cast<int>(2 * pairs), THREADS, P_SMEM_BYTES, s>>>(
-      ma, mb, mc, md, mm, g.epi, g.M, g.N, g.K, g.batch, g.sym ? 1 : 0, per_mat, staged, dev_err);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = P_SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc_gemm2_kernel<B_MN>, ma, mb, mc, md, mm, g.epi, g.M, g.N, g.K, g.batch,
+                            g.sym ? 1 : 0, per_mat, staged, dev_err);
 }
 
 }  // namespace
