@@ -179,3 +179,21 @@ def test_resident_small_kernel(dmuon_lib, shapes):
         w_apply = ora.apply_update(to64(Ws[i]), to64(Ob[i]), 0.02, 0.1)
         terms = np.abs(0.998 * to64(Ws[i])) + np.abs(0.02 * ora.rms_scale(r, c) * to64(Ob[i]))
         assert np.all(np.abs(to64(Wg[i]) - w_apply) <= np.abs(w_apply) * 2.0 ** -8 + terms * 1e-6), i
+
+
+def test_nonfinite_gradient_stays_in_its_matrix(dmuon_lib):
+    """A NaN in one gradient poisons that matrix's update only: the other
+    matrices of the same group and of other groups are computed as usual."""
+    shapes = [(256, 512)] * 3 + [(64, 256)] * 2
+    Ws, Gs, Ms = make_inputs(shapes, seed=61)
+    Gs[1] = Gs[1].clone()
+    Gs[1][7, 11] = float("nan")
+    Gs[3] = Gs[3].clone()
+    Gs[3][0, 0] = float("inf")
+    Os, _ = gpu_update(dmuon_lib, Gs, Ms)
+    for i in range(len(shapes)):
+        if i in (1, 3):
+            assert not torch.isfinite(Os[i]).all()
+            continue
+        _, Oo = oracle_update(Gs[i], Ms[i])
+        assert rel_fro(to64(Os[i]), Oo) <= BF16_TOL, i
