@@ -57,7 +57,8 @@ extern "C" {
 
 /* Status codes. */
 #define DMUON_OK 0
-#define DMUON_ERR_INVALID (-1)        /* null pointer, bad shape/count/steps, non-finite hyperparameter */
+#define DMUON_ERR_INVALID (-1)        /* null pointer, bad shape/count/steps, non-finite hyperparameter;
+                                         a side above 2^20 or more than 2^31 elements in one matrix */
 #define DMUON_ERR_DTYPE (-2)          /* unsupported dtype combination */
 #define DMUON_ERR_CUDA (-3)           /* a CUDA runtime/driver call failed */
 #define DMUON_ERR_OOM (-4)            /* workspace allocation failed or caller workspace too small */

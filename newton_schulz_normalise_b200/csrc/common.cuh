@@ -13,8 +13,9 @@
 namespace dmuon {
 
 // ---------------------------------------------------------------- errors
-// Device-side error word (per launch, in scratch); the host reads it after a
-// step when asked to.  Codes match the DMUON_ERR_* values in dmuon.h.
+// Device-side error code written to the word a launch is given (a mapped
+// host word the library checks at its next call, or a slot of the static
+// scratch).  Codes match the DMUON_ERR_* values in dmuon.h.
 constexpr int kErrTimeout = -5;
 
 // A wait on an mbarrier gives up after this long (ns).  No correct wait in
