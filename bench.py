@@ -395,6 +395,7 @@ def main():
             "roofline": {"bound": "tensor", "kernel": gemm_kernel, "achieved": round(ach, 1),
                          "peak": peak_tc, "unit": "TFLOP/s", "frac": round(ach / peak_tc, 4),
                          "traffic": traffic, "peak_source": f"{peaks['_source']} bf16_tflops (burst)",
+                         "frac_of_sustained": round(ach / peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]), 4),
                          "launches": gemm["launches"] // kt_steps,
                          "share_of_step": round(gemm["ms"] / kt_steps / ms_per_step, 3) if ms_per_step else None},
             "elementwise": {"bound": "hbm", "kernel": "momentum", "achieved": round(ew_gbs, 1),

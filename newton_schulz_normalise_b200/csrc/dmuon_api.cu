@@ -726,11 +726,20 @@ int autotune(DeviceCtx& c, const Chunk& ch, bool f32, const Hyper& h, int forced
 }
 
 
-// Host I/O pipeline: matrices per chunk (about 16 MB of gradients, at least
-// one matrix) and the 256-byte aligned stride of one staged gradient.
+// Host I/O pipeline: matrices per chunk (about DMUON_IO_CHUNK_MB, default 16,
+// MB of gradients, at least one matrix) and the 256-byte aligned stride of one
+// staged gradient.
+long long io_chunk_bytes() {
+  static const long long v = [] {
+    const char* b = getenv("DMUON_IO_CHUNK_MB");
+    const long long mb = b ? atoll(b) : 16;
+    return std::max(1LL, mb) << 20;
+  }();
+  return v;
+}
 int io_chunk(long long rows, long long cols, bool g_f32) {
   const long long bytes = rows * cols * (g_f32 ? 4 : 2);
-  const long long n = (16LL << 20) / std::max(bytes, 1LL);
+  const long long n = io_chunk_bytes() / std::max(bytes, 1LL);
   return static_cast<int>(std::max(1LL, std::min(n, 65535LL)));
 }
 size_t io_stride(long long rows, long long cols, bool g_f32) {

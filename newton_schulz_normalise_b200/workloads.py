@@ -75,6 +75,9 @@ WORKLOADS = {
         "skewed-shapes-bf16",
         ((64, 256, 512), (256, 1024, 128), (4096, 14336, 8), (14336, 4096, 8)),
         seed=3),
+    # the skewed set's tiny group on its own (the resident small-matrix kernel)
+    "batch512-64x256-bf16": Workload(
+        "batch512-64x256-bf16", ((64, 256, 512),), seed=3),
     # Llama-style 8B matrix set: 32 layers of q, k, v, o, gate, up, down
     "llama8b-matrices-bf16": Workload(
         "llama8b-matrices-bf16", _LLAMA8B_LAYER, seed=4, interleave=32),
