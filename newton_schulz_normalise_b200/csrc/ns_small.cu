@@ -58,6 +58,8 @@ __device__ __forceinline__ void get_row32(const uint8_t* tile, int r, int col, f
   }
 }
 
+__device__ __forceinline__ bool finite_scale(float s) { return s > 0.f && s <= 3.0e38f; }  // false for NaN and Inf
+
 struct SmallArgs {
   const __nv_bfloat16* X0;  // [cnt][m][ldx] unnormalised iterate (wide orientation)
   long long ldx;
@@ -108,13 +110,16 @@ __global__ void __launch_bounds__(128, 1) ns_small_kernel(const SmallArgs p, int
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  // X0 -> shared (zero rows outside the matrices)
+  // X0 -> shared (zero rows outside the matrices).  A matrix whose scale s
+  // is not a positive finite number (a NaN or Inf in its gradient) is loaded
+  // as zeros: the stacked products multiply across matrices (0 * NaN = NaN),
+  // so its values must not reach the shared tile; its output is NaN instead.
   const int chunks = xatoms * 8;  // 16-byte chunks per row (n padded to 64)
   for (int idx = tid; idx < SM_ROWS * chunks; idx += 128) {
     const int rr = idx / chunks, q = idx % chunks;
     const int jj = rr / p.mr, ii = rr % p.mr, ll = blockIdx.x * p.g + jj;
     uint4 u = make_uint4(0, 0, 0, 0);
-    if (ll < p.cnt && ii < p.m && q * 8 < p.n) {
+    if (ll < p.cnt && ii < p.m && q * 8 < p.n && finite_scale(p.s[ll])) {
       const __nv_bfloat16* src = p.X0 + static_cast<long long>(ll) * p.m * p.ldx + static_cast<long long>(ii) * p.ldx + q * 8;
       if (q * 8 + 8 <= p.n) {
         u = *reinterpret_cast<const uint4*>(src);
@@ -132,8 +137,11 @@ __global__ void __launch_bounds__(128, 1) ns_small_kernel(const SmallArgs p, int
   const uint32_t tmem = *tmem_slot;
   const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
   const uint32_t xs = smem_u32(Xs), as = smem_u32(As), ps = smem_u32(Ps);
-  const float sl = valid_row ? p.s[l] : 0.f;
-  const float s2l = valid_row ? p.s2[l] : 0.f;
+  // A poisoned matrix runs with zero scales, so its rows of X, A and P stay
+  // zero (its stacked neighbours see only zeros); its output is NaN.
+  const bool poisoned = valid_row && !finite_scale(p.s[l]);
+  const float sl = valid_row && !poisoned ? p.s[l] : 0.f;
+  const float s2l = valid_row && !poisoned ? p.s2[l] : 0.f;
   const int npad = xatoms * 64;
   uint32_t phase = 0;
   bool ok = true;
@@ -213,6 +221,10 @@ __global__ void __launch_bounds__(128, 1) ns_small_kernel(const SmallArgs p, int
         put_row32(Xs, r, c0, v);
       } else if (valid_row && c0 < p.n) {
         // fin: alpha 1 (the step's scale is applied above), per-matrix pointers
+        if (poisoned) {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) v[t] = __int_as_float(0x7fc00000);
+        }
         epilogue_row<32>(p.fin, l, i, c0, v, p.m, p.n);
       }
     }
@@ -227,7 +239,7 @@ __global__ void __launch_bounds__(128, 1) ns_small_kernel(const SmallArgs p, int
       float v[32];
       get_row32(Xs, r, c0, v);
 #pragma unroll
-      for (int t = 0; t < 32; ++t) v[t] *= sl;
+      for (int t = 0; t < 32; ++t) v[t] = poisoned ? __int_as_float(0x7fc00000) : v[t] * sl;
       epilogue_row<32>(p.fin, l, i, c0, v, p.m, p.n);
     }
   }
