@@ -277,9 +277,11 @@ def main():
     shapes = w.shapes()
     pdt = B.DMUON_BF16 if w.param_dtype == "bf16" else B.DMUON_F32
     opts = B.options(pdt, pdt)
+    # the parameter lists are marshalled once, as an optimiser loop would
+    tW, tG, tM = B.TensorList(Ws), B.TensorList(Gs), B.TensorList(Ms)
 
     def step():
-        B.dmuon_step_ex(Ws, Gs, Ms, w.lr, w.wd, w.mu, w.ns_steps, opts=opts, stream=stream)
+        B.dmuon_step_ex(tW, tG, tM, w.lr, w.wd, w.mu, w.ns_steps, opts=opts, stream=stream)
 
     def barrier():
         if ws > 1:
@@ -336,9 +338,10 @@ def main():
     hW = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in Ws]
     h2d = sum(x.numel() * x.element_size() for x in hG)
     d2h = sum(x.numel() * x.element_size() for x in hW)
+    thG, thW = B.TensorList(hG), B.TensorList(hW)
 
     def step_io():
-        B.dmuon_step_host_io(Ws, hG, Ms, w.lr, w.wd, w.mu, w.ns_steps, params_host_out=hW, opts=opts,
+        B.dmuon_step_host_io(tW, thG, tM, w.lr, w.wd, w.mu, w.ns_steps, params_host_out=thW, opts=opts,
                              stream=stream)
 
     for _ in range(2):  # plans of the host-I/O chunking

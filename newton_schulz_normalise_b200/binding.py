@@ -102,20 +102,58 @@ def _check(rc: int):
     return rc
 
 
-def _ptrs(tensors):
-    arr = (ctypes.c_void_p * max(len(tensors), 1))()
+def _ptrs_of(tensors):
+    return (ctypes.c_void_p * max(len(tensors), 1))(*[t.data_ptr() if t is not None else None for t in tensors])
+
+
+def _shapes_of(tensors):
+    flat = []
     for i, t in enumerate(tensors):
-        arr[i] = t.data_ptr() if t is not None else None
-    return arr
+        shape = t.shape
+        if len(shape) != 2 or not t.is_contiguous():
+            raise ValueError(f"matrix {i}: expected a contiguous 2-D tensor, got {tuple(shape)}")
+        flat += shape
+    return (ctypes.c_int64 * max(len(flat), 1))(*flat)
+
+
+class TensorList:
+    """A list of tensors marshalled once: the pointer array, the (rows, cols)
+    pairs and the dtype code, for a loop that passes the same tensors on
+    every step.  It holds references to the tensors; their storage must not
+    be reallocated while it is in use.  Any entry point that takes a list of
+    tensors takes a TensorList as well."""
+    __slots__ = ("tensors", "ptrs", "shapes", "dtype")
+
+    def __init__(self, tensors):
+        self.tensors = list(tensors)
+        self.ptrs = _ptrs_of(self.tensors)
+        self.shapes = _shapes_of(self.tensors) if self.tensors and self.tensors[0] is not None else None
+        self.dtype = _dtype_code(self.tensors[0]) if self.tensors and self.tensors[0] is not None else DMUON_BF16
+
+    def __len__(self):
+        return len(self.tensors)
+
+    def __getitem__(self, i):
+        return self.tensors[i]
+
+    def __iter__(self):
+        return iter(self.tensors)
+
+
+def _ptrs(tensors):
+    return tensors.ptrs if isinstance(tensors, TensorList) else _ptrs_of(tensors)
 
 
 def _shapes(tensors):
-    arr = (ctypes.c_int64 * max(2 * len(tensors), 1))()
-    for i, t in enumerate(tensors):
-        if t.dim() != 2 or not t.is_contiguous():
-            raise ValueError(f"matrix {i}: expected a contiguous 2-D tensor, got {tuple(t.shape)}")
-        arr[2 * i], arr[2 * i + 1] = t.shape
-    return arr
+    if isinstance(tensors, TensorList) and tensors.shapes is not None:
+        return tensors.shapes
+    return _shapes_of(tensors)
+
+
+def _list_dtype(tensors) -> int:
+    if isinstance(tensors, TensorList):
+        return tensors.dtype
+    return _dtype_code(tensors[0]) if len(tensors) else DMUON_BF16
 
 
 def _stream(stream):
@@ -165,8 +203,7 @@ def dmuon_step_ex(params, grads, momenta, lr, wd, mu, ns_steps=5, opts: Options 
     n = len(params)
     assert len(grads) == n and len(momenta) == n
     if opts is None:
-        opts = options(_dtype_code(params[0]) if n else DMUON_BF16,
-                       _dtype_code(grads[0]) if n else DMUON_BF16, **kw)
+        opts = options(_list_dtype(params), _list_dtype(grads), **kw)
     return _check(lib.dmuon_step_ex(_ptrs(params), _ptrs(grads), _ptrs(momenta), _shapes(grads), n,
                                     lr, wd, mu, ns_steps, ctypes.byref(opts), _stream(stream)))
 
@@ -180,8 +217,7 @@ def dmuon_step_host_io(params, grads_host, momenta, lr, wd, mu, ns_steps=5, para
     if params_host_out is not None:
         assert len(params_host_out) == n
     if opts is None:
-        opts = options(_dtype_code(params[0]) if n else DMUON_BF16,
-                       _dtype_code(grads_host[0]) if n else DMUON_BF16, **kw)
+        opts = options(_list_dtype(params), _list_dtype(grads_host), **kw)
     out = _ptrs(params_host_out) if params_host_out is not None else None
     return _check(lib.dmuon_step_host_io(_ptrs(params), _ptrs(grads_host), _ptrs(momenta), out, _shapes(params),
                                          n, lr, wd, mu, ns_steps, ctypes.byref(opts), _stream(stream)))
@@ -192,7 +228,7 @@ def dmuon_compute_update(grads, momenta, out, mu, ns_steps=5, opts: Options | No
     n = len(grads)
     assert len(momenta) == n and len(out) == n
     if opts is None:
-        dt = _dtype_code(grads[0]) if n else DMUON_BF16
+        dt = _list_dtype(grads)
         opts = options(dt, dt, **kw)
     return _check(lib.dmuon_compute_update(_ptrs(grads), _ptrs(momenta), _shapes(grads), n, mu, ns_steps,
                                            ctypes.byref(opts), _ptrs(out), _stream(stream)))

@@ -124,9 +124,10 @@ struct DeviceCtx {
   cudaStream_t side[kSide] = {};
   cudaEvent_t fork_ev = nullptr;
   cudaEvent_t side_done[kSide] = {};
-  // host I/O pipeline: copy-in and copy-out streams, two staging slots
+  // host I/O pipeline: copy-in and copy-out streams, kIoSlots staging slots
+  static constexpr int kIoSlots = 4;
   cudaStream_t cin = nullptr, cout = nullptr;
-  cudaEvent_t g_ready[2] = {}, g_free[2] = {}, w_done[2] = {}, io_done = nullptr;
+  cudaEvent_t g_ready[kIoSlots] = {}, g_free[kIoSlots] = {}, w_done[kIoSlots] = {}, io_done = nullptr;
 };
 
 std::mutex g_ctx_mu;
@@ -159,7 +160,7 @@ int get_ctx(DeviceCtx** out) {
     }
     CUDA_TRY(cudaStreamCreateWithFlags(&c->cin, cudaStreamNonBlocking));
     CUDA_TRY(cudaStreamCreateWithFlags(&c->cout, cudaStreamNonBlocking));
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < DeviceCtx::kIoSlots; ++i) {
       CUDA_TRY(cudaEventCreateWithFlags(&c->g_ready[i], cudaEventDisableTiming));
       CUDA_TRY(cudaEventCreateWithFlags(&c->g_free[i], cudaEventDisableTiming));
       CUDA_TRY(cudaEventCreateWithFlags(&c->w_done[i], cudaEventDisableTiming));
@@ -837,23 +838,34 @@ int run_step(Request& r) {
       load[best] += group_cost(k);
     }
   }
+  // Host I/O with every plan cached: consecutive chunks alternate between
+  // the caller's stream and side stream 1 (two scratch regions), so one
+  // chunk's kernels fill the SMs the other's last wave leaves idle while the
+  // copy streams run ahead through kIoSlots staging slots.
+  bool io_two = r.grads_host && !any_miss;
   std::vector<size_t> region_need(DeviceCtx::kSide + 1, 0);
   std::vector<size_t> region_off(DeviceCtx::kSide + 1, 0);
   auto layout_regions = [&] {
     std::fill(region_need.begin(), region_need.end(), 0);
     for (size_t k = 0; k < groups.size(); ++k) region_need[lane[k]] = std::max(region_need[lane[k]], needs[k]);
+    if (io_two) region_need[1] = std::max(region_need[1], region_need[0]);
     for (int i = 1; i <= DeviceCtx::kSide; ++i) region_off[i] = region_off[i - 1] + region_need[i - 1];
     ws_need = region_off[DeviceCtx::kSide] + region_need[DeviceCtx::kSide];
   };
   layout_regions();
   const size_t tables_bytes = align256(4 * sizeof(void*) * static_cast<size_t>(r.count));
-  if (g_ext_ptr && align256(ws_need) + tables_bytes > g_ext_bytes) {
+  const int io_slots = r.grads_host ? DeviceCtx::kIoSlots : 0;
+  auto ext_fits = [&] {
+    return align256(ws_need) + static_cast<size_t>(io_slots) * align256(stage_slot) + tables_bytes <= g_ext_bytes;
+  };
+  if (g_ext_ptr && !ext_fits()) {
     std::fill(lane.begin(), lane.end(), 0);  // a caller buffer too small for side streams: one stream
+    io_two = false;
     layout_regions();
   }
   // device pointer tables: 4 arrays of count pointers, after the chunk scratch
-  const size_t stage_off = align256(ws_need);  // host I/O: two gradient staging slots
-  const size_t tables_off = stage_off + 2 * align256(stage_slot);
+  const size_t stage_off = align256(ws_need);  // host I/O: the gradient staging slots
+  const size_t tables_off = stage_off + static_cast<size_t>(io_slots) * align256(stage_slot);
   const size_t total_ws = tables_off + tables_bytes;
   rc = ensure_ws(c, total_ws, r.s);
   if (rc) return rc;
@@ -895,7 +907,7 @@ int run_step(Request& r) {
         const int total = static_cast<int>(gr.idx.size());
         for (int c0 = 0; c0 < total; c0 += gr.chunk, ++j)
           for (int q = 0; q < std::min(gr.chunk, total - c0); ++q)
-            host[gstart[k] + c0 + q] = ws + stage_off + (j & 1) * align256(stage_slot) + q * stride;
+            host[gstart[k] + c0 + q] = ws + stage_off + (j % io_slots) * align256(stage_slot) + q * stride;
       }
     }
   }
@@ -911,6 +923,7 @@ int run_step(Request& r) {
   bool side_used[DeviceCtx::kSide] = {false, false, false};
   for (size_t k = 0; k < groups.size(); ++k)
     if (lane[k] > 0) side_used[lane[k] - 1] = true;
+  if (io_two) side_used[0] = true;
   const bool forked = side_used[0] || side_used[1] || side_used[2];
   if (forked) {
     CUDA_TRY(cudaEventRecord(c.fork_ev, r.s));
@@ -922,12 +935,13 @@ int run_step(Request& r) {
     Group& gr = groups[k];
     const Geo& g = geos[k];
     const int total = static_cast<int>(gr.idx.size());
-    const cudaStream_t gs = lane[k] == 0 ? r.s : c.side[lane[k] - 1];
     for (int c0 = 0; c0 < total; c0 += gr.chunk) {
+      const int ln = io_two ? (io_j & 1) : lane[k];
+      const cudaStream_t gs = ln == 0 ? r.s : c.side[ln - 1];
       Chunk ch;
       ch.g = &g;
       ch.cnt = std::min(gr.chunk, total - c0);
-      ch.base = ws + region_off[lane[k]];
+      ch.base = ws + region_off[ln];
       ch.nblk = momentum_partials(g.rows, g.cols, gr.chunk, c.num_sms);
       ch.L = make_layout(g, gr.chunk, ch.nblk);
       const int p = gstart[k] + c0;
@@ -940,11 +954,11 @@ int run_step(Request& r) {
         const int i = gr.idx[c0 + q];
         if (!aligned16(r.grads[i]) || !aligned16(r.moms[i])) ch.aligned = 0;
       }
-      const int slot = io_j & 1;
+      const int slot = r.grads_host ? io_j % io_slots : 0;
       if (r.grads_host) {
         // copy-in: this chunk's gradients into its staging slot, once the
-        // chunk two back has consumed that slot
-        if (io_j >= 2) CUDA_TRY(cudaStreamWaitEvent(c.cin, c.g_free[slot], 0));
+        // chunk io_slots back has consumed that slot
+        if (io_j >= io_slots) CUDA_TRY(cudaStreamWaitEvent(c.cin, c.g_free[slot], 0));
         const size_t bytes = static_cast<size_t>(g.rows) * g.cols * (g_f32 ? 4 : 2);
         for (int q = 0; q < ch.cnt; ++q)
           CUDA_TRY(cudaMemcpyAsync(host[p + q], r.grads[gr.idx[c0 + q]], bytes, cudaMemcpyHostToDevice, c.cin));

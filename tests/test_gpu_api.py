@@ -79,3 +79,19 @@ def test_timing_and_launch_count(dmuon_lib):
     assert kinds[1]["launches"] == 1 and kinds[1]["bytes"] == 512 * 512 * 4 * 12
     assert all(k["ms"] >= 0 for k in kinds)
     assert kinds[0]["flops"] > 0 or kinds[0]["launches"] == 0
+
+
+def test_tensor_list_step_is_bit_identical(dmuon_lib):
+    """A step through pre-marshalled TensorLists equals the plain-list step,
+    on two steps in a row (the marshalled arrays are reused)."""
+    shapes = [(64, 256)] * 4 + [(320, 200)] * 2
+    Ws, Gs, Ms = make_inputs(shapes, seed=71, m_std=1e-3)
+    W1, M1 = [w.clone() for w in Ws], [m.clone() for m in Ms]
+    W2, M2 = [w.clone() for w in Ws], [m.clone() for m in Ms]
+    tW, tG, tM = dmuon_lib.TensorList(W2), dmuon_lib.TensorList(Gs), dmuon_lib.TensorList(M2)
+    for _ in range(2):
+        dmuon_lib.dmuon_step(W1, Gs, M1, 0.02, 0.1, 0.95, 5)
+        dmuon_lib.dmuon_step(tW, tG, tM, 0.02, 0.1, 0.95, 5)
+    torch.cuda.synchronize()
+    for a, b in zip(W1 + M1, W2 + M2):
+        assert torch.equal(a, b)
