@@ -2,9 +2,10 @@
 //
 // Every Newton-Schulz product of the Muon step is one launch of this file's
 // kernels:
-//   A = X X^T        (both operands K-major rows of X; symmetric result)
-//   B = c A A + b A  (right operand as stored, MN-major; symmetric result)
-//   X' = B X + a X   (X is the MN-major right operand)
+//   A = X X^T             (both operands K-major rows of X; symmetric result)
+//   P = c A A + b A + a I (right operand as stored, MN-major; symmetric
+//                          result; the identity is the epilogue's diagonal add)
+//   X' = P X              (X is the MN-major right operand)
 // and the Gram-space products, which have the same operand forms.
 //
 // Two kernels, both persistent (one CTA per SM, 384 threads) and

@@ -78,6 +78,11 @@ int ns_small_group(int m);
 cudaError_t launch_ns_small(const void* X0, long long ldx, const float* s, const float* s2, int cnt, int m, int n,
                             int steps, float a, float b, float c, const Epilogue& fin, cudaStream_t st, int* err);
 
+// dst[l] <- src[l] for cnt buffers of `bytes` (a multiple of 16, every
+// pointer 16-byte aligned; host pointers must be mapped pinned memory).
+cudaError_t launch_copy_tables(const void* const* src, void* const* dst, long long bytes, int cnt, int num_sms,
+                               cudaStream_t st);
+
 // One-block kernel whose only mbarrier wait can never complete; it gives up
 // after limit_ns and records kErrTimeout in *err.
 cudaError_t launch_wait_selftest(int* err, unsigned long long limit_ns, cudaStream_t st);

@@ -268,7 +268,55 @@ __global__ void wait_selftest_kernel(int* err, unsigned long long limit_ns) {
     *reinterpret_cast<volatile int*>(err) = kErrTimeout;
 }
 
+// Copies cnt buffers of `bytes` each, dst[l] <- src[l], through the SMs.
+// Either side may be pinned host memory mapped into the device's address
+// space: the host I/O pipeline gathers gradients from, and scatters
+// parameters to, host memory this way with one launch per chunk instead of
+// one copy-engine transfer per matrix.  All pointers 16-byte aligned and
+// bytes % 16 == 0 (checked by the host).  Four 16-byte loads in flight per
+// thread cover the PCIe round trip; 128-thread blocks without shared memory
+// fit beside a persistent GEMM CTA on the same SM.
+constexpr int COPY_THREADS = 128;
+constexpr int COPY_UNROLL = 4;
+
+__global__ void __launch_bounds__(COPY_THREADS) copy_tables_kernel(const uint4* const* __restrict__ src,
+                                                                   uint4* const* __restrict__ dst, long long nvec) {
+  const uint4* s = src[blockIdx.y];
+  uint4* d = dst[blockIdx.y];
+  const long long stride = static_cast<long long>(gridDim.x) * COPY_THREADS * COPY_UNROLL;
+  for (long long base = static_cast<long long>(blockIdx.x) * COPY_THREADS * COPY_UNROLL + threadIdx.x; base < nvec;
+       base += stride) {
+    uint4 v[COPY_UNROLL];
+#pragma unroll
+    for (int u = 0; u < COPY_UNROLL; ++u) {
+      const long long i = base + static_cast<long long>(u) * COPY_THREADS;
+      if (i < nvec) v[u] = s[i];
+    }
+#pragma unroll
+    for (int u = 0; u < COPY_UNROLL; ++u) {
+      const long long i = base + static_cast<long long>(u) * COPY_THREADS;
+      if (i < nvec) d[i] = v[u];
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_copy_tables(const void* const* src, void* const* dst, long long bytes, int cnt, int num_sms,
+                               cudaStream_t st) {
+  if (cnt <= 0 || bytes <= 0) return cudaSuccess;
+  if (cnt > 65535 || bytes % 16 != 0) return cudaErrorInvalidValue;
+  const long long nvec = bytes / 16;
+  const long long per_block = static_cast<long long>(COPY_THREADS) * COPY_UNROLL;
+  long long bx = (static_cast<long long>(num_sms) * 2 + cnt - 1) / cnt;  // about two blocks per SM in all
+  const long long need = (nvec + per_block - 1) / per_block;
+  if (bx > need) bx = need;
+  if (bx < 1) bx = 1;
+  dim3 grid(static_cast<unsigned>(bx), cnt);
+  copy_tables_kernel<<<grid, COPY_THREADS, 0, st>>>(reinterpret_cast<const uint4* const*>(src),
+                                                    reinterpret_cast<uint4* const*>(dst), nvec);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_wait_selftest(int* err, unsigned long long limit_ns, cudaStream_t st) {
   wait_selftest_kernel<<<1, 32, 0, st>>>(err, limit_ns);

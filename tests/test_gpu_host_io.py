@@ -45,3 +45,37 @@ def test_host_io_without_copy_out(dmuon_lib):
     torch.cuda.synchronize()
     for a, b in zip(W, W_ref):
         assert (a.float() - b.float()).abs().max().item() <= 2 ** -7 * b.float().abs().max().item()
+
+
+def test_host_io_pageable_and_unaligned_buffers(dmuon_lib):
+    """Host buffers the copy kernel cannot take (pageable memory, a pinned
+    buffer at a 2-byte offset) go through copy-engine transfers; the result
+    is the same as with pinned, aligned buffers."""
+    shapes = [(256, 512)] * 4 + [(128, 384)] * 3
+    lr, wd, mu = 0.02, 0.1, 0.95
+    Ws, Gs, Ms = make_inputs(shapes, seed=79, m_std=1e-3)
+
+    def run(hG, hW):
+        W = [w.clone() for w in Ws]
+        M = [m.clone() for m in Ms]
+        for _ in range(2):
+            dmuon_lib.dmuon_step_host_io(W, hG, M, lr, wd, mu, 5, params_host_out=hW)
+        torch.cuda.synchronize()
+        return W, M
+
+    pinned = run([g.cpu().pin_memory() for g in Gs], [torch.empty(w.shape, dtype=w.dtype).pin_memory() for w in Ws])
+
+    def offset_pinned(t):  # pinned storage, data pointer 2 bytes past a 16-byte boundary
+        big = torch.empty(t.numel() + 8, dtype=t.dtype).pin_memory()
+        v = big[1:1 + t.numel()].view(t.shape)
+        v.copy_(t)
+        return v
+
+    hG_mixed = [g.cpu() for g in Gs[:4]] + [offset_pinned(g.cpu()) for g in Gs[4:]]
+    hW_mixed = [torch.empty(w.shape, dtype=w.dtype) for w in Ws[:4]] + [offset_pinned(w.cpu()) for w in Ws[4:]]
+    assert all(h.data_ptr() % 16 == 2 for h in hG_mixed[4:])
+    mixed = run(hG_mixed, hW_mixed)
+    for a, b in zip(pinned[0] + pinned[1], mixed[0] + mixed[1]):
+        assert torch.equal(a, b)
+    for i in range(len(shapes)):
+        assert torch.equal(hW_mixed[i], mixed[0][i].cpu()), i
