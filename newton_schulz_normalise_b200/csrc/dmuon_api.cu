@@ -857,7 +857,7 @@ int run_step(Request& r) {
       const Geo& g = geos[k];
       const int tl = groups[k].plan.tile;
       const long long tiles = tc_gemm_tiles(g.m, g.n, groups[k].chunk, tl, false);
-      const long long wave = tl == 512 ? c.num_sms / 2 : c.num_sms;
+      const long long wave = tl >= 512 ? c.num_sms / 2 : c.num_sms;
       if (groups[k].idx.size() <= static_cast<size_t>(groups[k].chunk) && tiles < 2 * wave)
         small.push_back(static_cast<int>(k));
     }

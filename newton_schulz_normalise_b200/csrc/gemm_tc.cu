@@ -122,7 +122,7 @@ __device__ __forceinline__ void store_tile_staged(const Epilogue& e, const CUten
     const uint32_t b = st.it % NRING;
     uint8_t* buf = wstg + b * WBOX;
     uint8_t* mbuf = wstg + (NRING + (st.it & 1)) * WBOX;
-    const bool live = col < N;
+    const bool live = col < N && row0w < M;  // a 32-row box wholly below the result is not stored
     if (lane == 0) {
       bulk_wait_read<1>();  // the stores issued from these buffers two chunks ago have read them
       if (has_c && live) {
@@ -731,7 +731,8 @@ cudaError_t launch_tc_gemm(const TcGemm& g, cudaStream_t s, int* dev_err, int nu
   TcGemm h = g;
   h.epi.sym = g.sym ? 1 : 0;
   const bool mn = !g.b_kmajor;
-  if (g.tile == 512) return mn ? launch_pair<true>(h, s, dev_err, num_sms) : launch_pair<false>(h, s, dev_err, num_sms);
+  if (g.tile == 512)
+    return mn ? launch_pair<true>(h, s, dev_err, num_sms) : launch_pair<false>(h, s, dev_err, num_sms);
   if (g.tile == 128)
     return mn ? launch_one<128, true>(h, s, dev_err, num_sms) : launch_one<128, false>(h, s, dev_err, num_sms);
   return mn ? launch_one<256, true>(h, s, dev_err, num_sms) : launch_one<256, false>(h, s, dev_err, num_sms);

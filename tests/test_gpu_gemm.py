@@ -66,13 +66,14 @@ def test_gemm_without_addend_and_alpha(dmuon_lib):
     assert torch.allclose(D.float(), D.float().transpose(1, 2), rtol=2 ** -7, atol=1e-3)
 
 
-def test_gemm_deterministic(dmuon_lib):
+@pytest.mark.parametrize("tile", [256, 512])
+def test_gemm_deterministic(dmuon_lib, tile):
     A = torch.randn(4, 512, 1024, device="cuda").bfloat16()
     B = torch.randn(4, 1024, 768, device="cuda").bfloat16()
     D1 = torch.empty(4, 512, 768, device="cuda", dtype=torch.bfloat16)
     D2 = torch.empty_like(D1)
-    dmuon_lib.dmuon_gemm_bf16(A, B, D1, b_kmajor=False)
-    dmuon_lib.dmuon_gemm_bf16(A, B, D2, b_kmajor=False)
+    dmuon_lib.dmuon_gemm_bf16(A, B, D1, b_kmajor=False, tile=tile)
+    dmuon_lib.dmuon_gemm_bf16(A, B, D2, b_kmajor=False, tile=tile)
     torch.cuda.synchronize()
     assert torch.equal(D1, D2)
 

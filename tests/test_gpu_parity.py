@@ -201,3 +201,25 @@ def test_nonfinite_gradient_stays_in_its_matrix(dmuon_lib, variant):
             continue
         _, Oo = oracle_update(Gs[i], Ms[i])
         assert rel_fro(to64(Os[i]), Oo) <= BF16_TOL, i
+
+
+@pytest.mark.parametrize("tile", ["256", "512"])
+def test_forced_tile_matches_oracle(dmuon_lib, monkeypatch, tile):
+    """The Muon update with the autotuner restricted to one tile shape
+    (DMUON_TILE): one CTA per 128 x 256 tile, and the CTA pair.  m > 256,
+    odd and even numbers of 256-row tile rows, ragged edges."""
+    shapes = [(1024, 1024)] * 2 + [(600, 1000)] * 2 + [(1000, 520)] + [(768, 768)]
+    Ws, Gs, Ms = make_inputs(shapes, seed=83, m_std=1e-3)
+    monkeypatch.setenv("DMUON_TILE", tile)
+    dmuon_lib.dmuon_cache_clear()
+    try:
+        Os, Bn = gpu_update(dmuon_lib, Gs, Ms, variant="direct")
+        plans = dmuon_lib.dmuon_cache_entries()
+    finally:
+        dmuon_lib.dmuon_cache_clear()
+    assert all(e.split()[5] == tile for e in plans), plans
+    for i in range(len(shapes)):
+        _, Oo = oracle_update(Gs[i], Ms[i])
+        e = rel_fro(to64(Os[i]), Oo)
+        assert e <= BF16_TOL, (shapes[i], tile, e)
+        check_momentum(Bn[i], Gs[i], Ms[i], 0.95)
