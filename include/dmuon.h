@@ -120,10 +120,15 @@ int dmuon_step_ex(void* const* params, const void* const* grads, void* const* mo
  * dmuon_step_host_io -- dmuon_step_ex for gradients that live in HOST memory
  * (e.g. reduced or offloaded on the CPU), with the updated parameters copied
  * back to host memory.  The call splits every shape group into chunks of
- * about 16 MB of gradients and pipelines them over two internal copy
- * streams: chunk i+1's gradients travel host->device while chunk i is
- * computed and chunk i-1's parameters travel device->host, through two
- * staging slots in the scratch.
+ * about 16 MB of gradients (DMUON_IO_CHUNK_MB) and pipelines them over two
+ * internal copy streams: later chunks' gradients travel host->device
+ * (through four staging slots in the scratch) while a chunk is computed and
+ * earlier chunks' parameters travel device->host.  Once every plan is
+ * cached, consecutive chunks alternate between `stream` and an internal
+ * compute stream.  Matrices of at most 256 KB whose host buffers are pinned
+ * and 16-byte aligned are copied by a kernel that reads and writes the
+ * mapped host memory, one launch per chunk; other matrices take one
+ * copy-engine transfer each (DMUON_IO_COPY=dma|kernel forces one kind).
  *   params[i]          device, updated in place (as dmuon_step).
  *   grads_host[i]      host, rows_i x cols_i row-major; pinned (page-locked)
  *                      memory for the copies to run asynchronously.

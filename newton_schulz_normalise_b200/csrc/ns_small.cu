@@ -14,7 +14,12 @@
 //   X' = P X        (128 x n, K = 128)   acts on each matrix separately.
 // X, A and P live in the 128-byte-swizzled K-major layout that the MMA reads
 // directly; the same bytes serve as the MN-major right operand (a K-major
-// matrix with rows = k is the MN-major layout of its row-major self).
+// matrix with rows = k is the MN-major layout of its row-major self).  P
+// overwrites A in place (each thread reads its row of A before writing the
+// same row of P), and the three products of a step run one after another,
+// so each accumulates from TMEM column 0: a CTA needs max(128, n) columns.
+// For n <= 256 that is 97 KB of shared memory and 256 TMEM columns, so two
+// CTAs share an SM and each hides the other's latency.
 // One thread issues the MMAs; every wait is bounded (2 s).
 #include <mutex>
 
@@ -84,14 +89,16 @@ __device__ __forceinline__ void issue(uint32_t d_tmem, uint32_t a_base, uint32_t
   umma_commit(bar);
 }
 
-__global__ void __launch_bounds__(128, 1) ns_small_kernel(const SmallArgs p, int* err) {
+__host__ __device__ constexpr int small_tmem_cols(int n) { return n <= 128 ? 128 : (n <= 256 ? 256 : 512); }
+
+__global__ void __launch_bounds__(128, 2) ns_small_kernel(const SmallArgs p, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int xatoms = (p.n + 63) / 64;
   uint8_t* Xs = smem;                      // 128 x n, xatoms atoms
-  uint8_t* As = Xs + xatoms * ATOM;        // 128 x 128
-  uint8_t* Ps = As + 2 * ATOM;             // 128 x 128
-  uint64_t* bar = reinterpret_cast<uint64_t*>(Ps + 2 * ATOM);
+  uint8_t* As = Xs + xatoms * ATOM;        // 128 x 128: A, then P in place
+  uint8_t* Ps = As;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(As + 2 * ATOM);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -107,7 +114,7 @@ __global__ void __launch_bounds__(128, 1) ns_small_kernel(const SmallArgs p, int
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, small_tmem_cols(p.n));
     tmem_relinquish();
   }
   // X0 -> shared (zero rows outside the matrices).  A matrix whose scale s
@@ -170,7 +177,7 @@ __global__ void __launch_bounds__(128, 1) ns_small_kernel(const SmallArgs p, int
     __syncthreads();
     tc_fence_after();
     // ---- P = c A A + b A + a I
-    if (tid == 0) issue(tmem + 256, as, as, true, SM_ROWS, SM_ROWS, bar);
+    if (tid == 0) issue(tmem, as, as, true, SM_ROWS, SM_ROWS, bar);
     ok = mbar_wait(bar, phase, abort);
     phase ^= 1;
     if (!__syncthreads_and(ok)) break;
@@ -178,8 +185,8 @@ __global__ void __launch_bounds__(128, 1) ns_small_kernel(const SmallArgs p, int
 #pragma unroll 1
     for (int c0 = 0; c0 < SM_ROWS; c0 += 32) {
       float v[32], av[32];
-      tmem_ld_32cols(trow + 256 + c0, v);
-      get_row32(As, r, c0, av);
+      tmem_ld_32cols(trow + c0, v);
+      get_row32(As, r, c0, av);  // this row of A, then the same row of P over it
 #pragma unroll
       for (int t = 0; t < 32; ++t) v[t] = p.c * v[t] + p.b * av[t] + ((c0 + t) == r ? p.a : 0.f);
       put_row32(Ps, r, c0, v);
@@ -247,7 +254,7 @@ __global__ void __launch_bounds__(128, 1) ns_small_kernel(const SmallArgs p, int
   if (*abort && tid == 0 && err) *reinterpret_cast<volatile int*>(err) = kErrTimeout;
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, small_tmem_cols(p.n));
   }
 }
 
@@ -285,8 +292,8 @@ cudaError_t launch_ns_small(const void* X0, long long ldx, const float* s, const
   p.fin.beta = 0.f;
   p.fin.C = nullptr;
   const int xatoms = (n + 63) / 64;                     // X: up to 8 atoms (n <= 512)
-  const int smem = (xatoms + 4) * ATOM + 1024 + 64;      // + A and P (2 atoms each), alignment, barrier
-  constexpr int kMaxSmem = (8 + 4) * ATOM + 1024 + 64;   // 197,696 bytes
+  const int smem = (xatoms + 2) * ATOM + 1024 + 64;      // + A / P (2 atoms), alignment, barrier
+  constexpr int kMaxSmem = (8 + 2) * ATOM + 1024 + 64;   // 164,928 bytes
   static std::once_flag once;
   static cudaError_t attr = cudaSuccess;
   std::call_once(once, [] {
