@@ -1,4 +1,5 @@
-"""fp64 CPU oracle of the Muon / DMuon step.
+"""fp64 CPU oracles of the Muon / DMuon step (``muon_oracle``) and of the
+AdamW step for non-matrix parameters (``adamw_oracle``).
 
 Test infrastructure only: imported by ``tests/``, ``__graft_entry__.smoke()``
 and ``bench.py``'s CPU-baseline / reference legs, never by the library.
