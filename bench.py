@@ -159,7 +159,24 @@ def cpu_baseline(w, budget_s=12.0):
         "sample": f"{done} of {len(shapes)} matrices timed one by one (fp64 numpy, BLAS on "
                   f"{cores} threads), mean per shape x count",
         "cpu": _cpu_model(),
+        "adamw": adamw_oracle_time(),
     }
+
+
+def adamw_oracle_time():
+    """The fp64 AdamW oracle on 1/16 of the bench's AdamW set (3144 rows of
+    the 50304 x 1024 table plus 6 of the 96 vectors), scaled to the whole set."""
+    import numpy as np
+    import oracle.adamw_oracle as aora
+    rng = np.random.default_rng(5)
+    parts = [rng.standard_normal((3144, 1024)) * 0.02] + [rng.standard_normal(1024) * 0.02 for _ in range(6)]
+    t0 = time.perf_counter()
+    for p in parts:
+        g = p * 0.05
+        aora.adamw_step(p, g, np.zeros_like(p), np.zeros_like(p), 1e-3, 0.9, 0.95, 1e-8, 0.1, 4)
+    dt = time.perf_counter() - t0
+    return {"value": dt * 16 * 1e3, "unit": "ms", "kind": "oracle",
+            "sample": "1/16 of the 50304x1024 + 96x1024 set (fp64 numpy), scaled by 16"}
 
 
 def _cpu_model():
@@ -237,6 +254,35 @@ def profile_traffic(kernel_file: Path):
         if line.startswith("traffic_bytes_per_launch:"):
             traffic = float(line.split(":", 1)[1].strip())
     return traffic if src == sha else None
+
+
+def adamw_measure(dev, stream, torch_dtype, iters=20):
+    """Device time of one dmuon_adamw_step over an embedding-sized set of
+    non-matrix parameters; returns ms, GB/s of algorithmic bytes, element
+    count and bytes per element."""
+    import torch
+    from newton_schulz_normalise_b200 import binding as B
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5)
+    shapes = [(50304, 1024)] + [(1024,)] * 96
+    P = [(torch.randn(s, device=dev, generator=gen) * 0.02).to(torch_dtype) for s in shapes]
+    G = [(torch.randn(s, device=dev, generator=gen) * 1e-3).to(torch_dtype) for s in shapes]
+    M = [torch.zeros(s, device=dev) for s in shapes]
+    V = [torch.zeros(s, device=dev) for s in shapes]
+    tP, tG, tM, tV = B.TensorList(P), B.TensorList(G), B.TensorList(M), B.TensorList(V)
+    for t in range(1, 4):
+        B.dmuon_adamw_step(tP, tG, tM, tV, 1e-3, 0.9, 0.95, 1e-8, 0.1, t, stream=stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for t in range(4, 4 + iters):
+        B.dmuon_adamw_step(tP, tG, tM, tV, 1e-3, 0.9, 0.95, 1e-8, 0.1, t, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / iters
+    n = sum(p.numel() for p in P)
+    bpe = 22 if torch_dtype == torch.bfloat16 else 32
+    return {"ms": ms, "gbs": n * bpe / (ms * 1e-3) / 1e9, "elements": n, "bpe": bpe}
 
 
 def main():
@@ -357,6 +403,13 @@ def main():
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
+    # ---------------- AdamW on the non-matrix parameters that train beside Muon
+    # (a separate measurement, outside the step above): one 50304 x 1024
+    # embedding table plus 96 vectors of 1024, in the workload's dtype, fp32
+    # moments; 1.2 GB per launch (bf16) > L2.  Times dmuon_adamw_step alone.
+    aw = adamw_measure(dev, stream, torch_dtype=wl.torch_dtype(w.param_dtype))
+    del hG, hW, thG, thW
+
     # ---------------- reduce over ranks (max), report on rank 0
     ms_max, e2e_max = reduce_max([ms, e2e_ms], ws, device=dev)
     ms_per_step = ms_max / args.steps
@@ -404,6 +457,10 @@ def main():
             "elementwise": {"bound": "hbm", "kernel": "momentum", "achieved": round(ew_gbs, 1),
                             "peak": peaks["hbm_gbs"], "unit": "GB/s",
                             "frac": round(ew_gbs / peaks["hbm_gbs"], 4)},
+            "adamw": {"bound": "hbm", "kernel": "adamw_kernel", "achieved": round(aw["gbs"], 1),
+                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(aw["gbs"] / peaks["hbm_gbs"], 4),
+                      "ms": round(aw["ms"], 4), "elements": aw["elements"], "bytes_per_element": aw["bpe"],
+                      "set": "50304x1024 embedding + 96 x 1024 vectors"},
             "e2e": {"value": round(job_value(e2e_max, 1, ws), 4), "unit": "ms", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches * args.steps,

@@ -235,6 +235,38 @@ void dmuon_timing_reset(void);
 int dmuon_timing_get(int kind, int64_t* launches, double* ms, double* flops, double* bytes);
 
 /*
+ * dmuon_adamw_step -- one AdamW step for the parameters that are not
+ * matrices.  "DeepSpeed 現已支援 Muon Optimizer" (setupai.cc), section
+ * 技術深入: Muon trains the matrix parameters (2-D weights, and convolution
+ * filters once flattened) while AdamW trains the rest, such as embeddings,
+ * biases and the final classification layer.  The pages give no AdamW
+ * formula; this is the published algorithm with decoupled weight decay and
+ * bias correction, per element, in fp32:
+ *   m = beta1 m + (1 - beta1) g,   v = beta2 v + (1 - beta2) g^2
+ *   p = (1 - lr wd) p - lr (m / (1 - beta1^step)) / (sqrt(v / (1 - beta2^step)) + eps)
+ * with one rounding of p to its dtype.  All tensors run in one launch.
+ *   params[i]      device, numels[i] elements, dtype `dtype` (DMUON_BF16 or
+ *                  DMUON_F32), updated in place.
+ *   grads[i]       device, same dtype and size, read only.
+ *   exp_avg[i], exp_avg_sq[i]
+ *                  device fp32 moment buffers (start at zero), in place.
+ *   numels[i]      element count (>= 0; 0 skips the tensor).  Any layout:
+ *                  the four buffers of a tensor are walked as flat arrays.
+ *   step           1 for the first step, then 2, 3, ... (bias correction).
+ * The pointer arrays are host memory, read during the call.  Asynchronous
+ * on `stream`.  Errors (before any launch, nothing modified):
+ * DMUON_ERR_INVALID for a null pointer, numel < 0, step < 1, a non-finite
+ * hyperparameter, beta outside [0, 1) or eps < 0; DMUON_ERR_DTYPE for
+ * another dtype; DMUON_ERR_OOM if the device tables cannot be allocated.
+ * 16-byte aligned buffers take a 4-element vector path; others are handled
+ * element by element.
+ */
+int dmuon_adamw_step(void* const* params, const void* const* grads, float* const* exp_avg,
+                     float* const* exp_avg_sq, const int64_t* numels, int count, float lr,
+                     float beta1, float beta2, float eps, float wd, int64_t step, int dtype,
+                     void* stream);
+
+/*
  * dmuon_selftest_wait -- checks the device-side failure path: launches a
  * one-block kernel whose mbarrier wait nothing completes, with a limit of
  * limit_ms (1..2000).  The kernel gives up, records the timeout in the

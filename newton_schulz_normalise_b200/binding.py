@@ -33,7 +33,7 @@ EXPORTS = (
     "dmuon_cache_size", "dmuon_cache_entry", "dmuon_set_workspace", "dmuon_workspace_size",
     "dmuon_timing_enable", "dmuon_timing_reset", "dmuon_timing_get", "dmuon_launch_count",
     "dmuon_last_error", "dmuon_version", "dmuon_compute_update_noalloc", "dmuon_step_host_io",
-    "dmuon_selftest_wait",
+    "dmuon_selftest_wait", "dmuon_adamw_step",
 )
 
 
@@ -81,6 +81,7 @@ def _load() -> ctypes.CDLL:
         "dmuon_compute_update_noalloc": (I, [P, P, I64, I64, F, I, ctypes.POINTER(Options), P, P]),
         "dmuon_step_host_io": (I, [PP, PP, PP, PP, PI64, I, F, F, F, I, ctypes.POINTER(Options), P]),
         "dmuon_selftest_wait": (I, [I, P]),
+        "dmuon_adamw_step": (I, [PP, PP, PP, PP, PI64, I, F, F, F, F, F, I64, I, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -127,7 +128,10 @@ class TensorList:
     def __init__(self, tensors):
         self.tensors = list(tensors)
         self.ptrs = _ptrs_of(self.tensors)
-        self.shapes = _shapes_of(self.tensors) if self.tensors and self.tensors[0] is not None else None
+        # (rows, cols) pairs when every tensor is a contiguous matrix (the Muon
+        # entry points need them); AdamW lists of any rank leave them unset
+        mats = all(t is not None and t.dim() == 2 and t.is_contiguous() for t in self.tensors)
+        self.shapes = _shapes_of(self.tensors) if self.tensors and mats else None
         self.dtype = _dtype_code(self.tensors[0]) if self.tensors and self.tensors[0] is not None else DMUON_BF16
 
     def __len__(self):
@@ -247,6 +251,21 @@ def dmuon_compute_update_noalloc(grad, momentum, out, mu, ns_steps=5, opts: Opti
     return _check(lib.dmuon_compute_update_noalloc(grad.data_ptr(), momentum.data_ptr(), rows, cols, mu,
                                                    ns_steps, ctypes.byref(opts), out.data_ptr(),
                                                    _stream(stream)))
+
+
+def dmuon_adamw_step(params, grads, exp_avg, exp_avg_sq, lr, beta1, beta2, eps, wd, step, stream=None):
+    """One AdamW step over lists of tensors (any shapes, contiguous): bf16 or
+    fp32 params and grads (one dtype for the call), fp32 moment buffers."""
+    n = len(params)
+    assert len(grads) == n and len(exp_avg) == n and len(exp_avg_sq) == n
+    for group in (params, grads, exp_avg, exp_avg_sq):
+        for t in group:
+            if not t.is_contiguous():
+                raise ValueError("AdamW tensors must be contiguous")
+    numels = (ctypes.c_int64 * max(n, 1))(*[t.numel() for t in params])
+    return _check(lib.dmuon_adamw_step(_ptrs(params), _ptrs(grads), _ptrs(exp_avg), _ptrs(exp_avg_sq), numels, n,
+                                       lr, beta1, beta2, eps, wd, int(step), _list_dtype(params),
+                                       _stream(stream)))
 
 
 def dmuon_gemm_bf16(A, B, D, alpha=1.0, beta=0.0, C=None, b_kmajor=True, tile=0, sym=False, stream=None):

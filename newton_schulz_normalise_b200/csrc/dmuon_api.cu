@@ -124,6 +124,11 @@ struct DeviceCtx {
   cudaStream_t side[kSide] = {};
   cudaEvent_t fork_ev = nullptr;
   cudaEvent_t side_done[kSide] = {};
+  // AdamW pointer / size tables (device) and the event after the last AdamW launch
+  void* adam_tab = nullptr;
+  size_t adam_cap = 0;
+  cudaEvent_t adam_done = nullptr;
+  bool adam_used = false;
   // host I/O pipeline: copy-in and copy-out streams, kIoSlots staging slots
   static constexpr int kIoSlots = 4;
   cudaStream_t cin = nullptr, cout = nullptr;
@@ -166,6 +171,7 @@ int get_ctx(DeviceCtx** out) {
       CUDA_TRY(cudaEventCreateWithFlags(&c->w_done[i], cudaEventDisableTiming));
     }
     CUDA_TRY(cudaEventCreateWithFlags(&c->io_done, cudaEventDisableTiming));
+    CUDA_TRY(cudaEventCreateWithFlags(&c->adam_done, cudaEventDisableTiming));
     CUDA_TRY(cudaHostAlloc(reinterpret_cast<void**>(&c->err_host), sizeof(int), cudaHostAllocMapped));
     *c->err_host = 0;
     CUDA_TRY(cudaHostGetDevicePointer(reinterpret_cast<void**>(&c->err_dev), c->err_host, 0));
@@ -1301,6 +1307,104 @@ int dmuon_gemm_bf16(const void* A, int64_t lda, int64_t sa, const void* B, int64
   cudaError_t err = launch_k(KIND_TC_GEMM, 2.0 * M * N * static_cast<double>(K) * batch * frac, 0.0, s,
                              [&] { return launch_tc_gemm(t, s, cp->err_dev, cp->num_sms); });
   if (err != cudaSuccess) return fail(DMUON_ERR_CUDA, "gemm launch: %s", cudaGetErrorString(err));
+  return DMUON_OK;
+}
+
+int dmuon_adamw_step(void* const* params, const void* const* grads, float* const* exp_avg, float* const* exp_avg_sq,
+                     const int64_t* numels, int count, float lr, float beta1, float beta2, float eps, float wd,
+                     int64_t step, int dtype, void* stream) {
+  t_err.clear();
+  if (count < 0) return fail(DMUON_ERR_INVALID, "count < 0");
+  if (count == 0) return DMUON_OK;
+  if (!params || !grads || !exp_avg || !exp_avg_sq || !numels) return fail(DMUON_ERR_INVALID, "null pointer array");
+  if (dtype != DMUON_BF16 && dtype != DMUON_F32) return fail(DMUON_ERR_DTYPE, "dtype must be BF16 or F32");
+  if (step < 1) return fail(DMUON_ERR_INVALID, "step counts from 1 (got %lld)", static_cast<long long>(step));
+  const float hs[] = {lr, beta1, beta2, eps, wd};
+  for (float v : hs)
+    if (!std::isfinite(v)) return fail(DMUON_ERR_INVALID, "non-finite hyperparameter");
+  if (beta1 < 0.f || beta1 >= 1.f || beta2 < 0.f || beta2 >= 1.f || eps < 0.f)
+    return fail(DMUON_ERR_INVALID, "betas must be in [0, 1) and eps >= 0");
+  // live tensors (numel > 0) and their chunk offsets
+  std::vector<int> live;
+  std::vector<long long> starts;
+  long long chunks = 0;
+  bool aligned = true;
+  for (int i = 0; i < count; ++i) {
+    if (numels[i] < 0) return fail(DMUON_ERR_INVALID, "tensor %d has numel %lld", i, static_cast<long long>(numels[i]));
+    if (numels[i] == 0) continue;
+    if (!params[i] || !grads[i] || !exp_avg[i] || !exp_avg_sq[i]) return fail(DMUON_ERR_INVALID, "null pointer for tensor %d", i);
+    aligned = aligned && aligned16(params[i]) && aligned16(grads[i]) && aligned16(exp_avg[i]) && aligned16(exp_avg_sq[i]);
+    live.push_back(i);
+    starts.push_back(chunks);
+    chunks += adamw_chunks(numels[i]);
+  }
+  const int n = static_cast<int>(live.size());
+  if (n == 0) return DMUON_OK;
+  if (chunks > 0x7fffffffLL) return fail(DMUON_ERR_INVALID, "too many elements for one launch");
+  DeviceCtx* cp = nullptr;
+  int rc = get_ctx(&cp);
+  if (rc) return rc;
+  DeviceCtx& c = *cp;
+  std::lock_guard<std::mutex> lk(c.mu);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // tables: P, G, M, V pointers, chunk starts, numels (8 bytes each)
+  std::vector<void*> host(6 * static_cast<size_t>(n));
+  for (int k = 0; k < n; ++k) {
+    const int i = live[k];
+    host[k] = params[i];
+    host[n + k] = const_cast<void*>(grads[i]);
+    host[2 * n + k] = exp_avg[i];
+    host[3 * n + k] = exp_avg_sq[i];
+    host[4 * n + k] = reinterpret_cast<void*>(static_cast<intptr_t>(starts[k]));
+    host[5 * n + k] = reinterpret_cast<void*>(static_cast<intptr_t>(numels[i]));
+  }
+  const size_t bytes = host.size() * sizeof(void*);
+  if (c.adam_used) CUDA_TRY(cudaStreamWaitEvent(s, c.adam_done, 0));  // the previous launch has read the tables
+  if (bytes > c.adam_cap) {
+    if (fault_alloc()) return fail(DMUON_ERR_OOM, "injected allocation failure (DMUON_FAULT=alloc)");
+    if (c.adam_tab) {
+      CUDA_TRY(cudaStreamSynchronize(s));
+      CUDA_TRY(cudaFree(c.adam_tab));
+      c.adam_tab = nullptr;
+      c.adam_cap = 0;
+    }
+    const size_t cap = std::max<size_t>(bytes, 64 << 10);
+    if (cudaMalloc(&c.adam_tab, cap) != cudaSuccess) {
+      cudaGetLastError();
+      return fail(DMUON_ERR_OOM, "AdamW tables: cannot allocate %zu bytes", cap);
+    }
+    c.adam_cap = cap;
+  }
+  rc = upload_tables(c, host, c.adam_tab, s);
+  if (rc) return rc;
+  void** tab = static_cast<void**>(c.adam_tab);
+  AdamwArgs a{};
+  a.P = tab;
+  a.G = tab + n;
+  a.M = reinterpret_cast<float* const*>(tab + 2 * n);
+  a.V = reinterpret_cast<float* const*>(tab + 3 * n);
+  a.chunk_start = reinterpret_cast<const long long*>(tab + 4 * n);
+  a.numel = reinterpret_cast<const long long*>(tab + 5 * n);
+  a.count = n;
+  a.p_f32 = dtype == DMUON_F32 ? 1 : 0;
+  a.aligned = aligned ? 1 : 0;
+  a.lr = lr;
+  a.beta1 = beta1;
+  a.beta2 = beta2;
+  a.eps = eps;
+  a.omb1 = static_cast<float>(1.0 - static_cast<double>(beta1));
+  a.omb2 = static_cast<float>(1.0 - static_cast<double>(beta2));
+  a.decay = static_cast<float>(1.0 - static_cast<double>(lr) * static_cast<double>(wd));
+  a.bc1 = static_cast<float>(1.0 - std::pow(static_cast<double>(beta1), static_cast<double>(step)));
+  a.bc2 = static_cast<float>(1.0 - std::pow(static_cast<double>(beta2), static_cast<double>(step)));
+  if (!(a.bc1 > 0.f) || !(a.bc2 > 0.f)) return fail(DMUON_ERR_INVALID, "bias correction 1 - beta^t is not positive");
+  long long elems = 0;
+  for (int k = 0; k < n; ++k) elems += numels[live[k]];
+  const double ebytes = static_cast<double>(elems) * (dtype == DMUON_F32 ? 32.0 : 22.0);
+  cudaError_t e = launch_k(KIND_EW, 0.0, ebytes, s, [&] { return launch_adamw(a, chunks, s); });
+  if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "AdamW kernel: %s", cudaGetErrorString(e));
+  CUDA_TRY(cudaEventRecord(c.adam_done, s));
+  c.adam_used = true;
   return DMUON_OK;
 }
 

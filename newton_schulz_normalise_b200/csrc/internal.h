@@ -78,6 +78,27 @@ int ns_small_group(int m);
 cudaError_t launch_ns_small(const void* X0, long long ldx, const float* s, const float* s2, int cnt, int m, int n,
                             int steps, float a, float b, float c, const Epilogue& fin, cudaStream_t st, int* err);
 
+// AdamW over `count` tensors in one launch (see kernels_ew.cu).  Tables are
+// device arrays; chunk_start[t] is the first chunk of tensor t (prefix sums of
+// adamw_chunks(numel)), numel[t] its element count (> 0).
+struct AdamwArgs {
+  void* const* P;           // params, bf16 or fp32 (p_f32), updated in place
+  const void* const* G;     // grads, same dtype as P
+  float* const* M;          // first moments, fp32, in place
+  float* const* V;          // second moments, fp32, in place
+  const long long* chunk_start;
+  const long long* numel;
+  int count;
+  int p_f32;
+  int aligned;              // every P/G/M/V base 16-byte aligned: 4-element vectors
+  float lr, beta1, beta2, eps;
+  float omb1, omb2;         // 1 - beta1, 1 - beta2
+  float decay;              // 1 - lr * wd
+  float bc1, bc2;           // 1 - beta1^t, 1 - beta2^t
+};
+long long adamw_chunks(long long numel);
+cudaError_t launch_adamw(const AdamwArgs& a, long long total_chunks, cudaStream_t st);
+
 // dst[l] <- src[l] for cnt buffers of `bytes` (a multiple of 16, every
 // pointer 16-byte aligned; host pointers must be mapped pinned memory).
 cudaError_t launch_copy_tables(const void* const* src, void* const* dst, long long bytes, int cnt, int num_sms,

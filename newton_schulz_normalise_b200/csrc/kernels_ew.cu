@@ -300,7 +300,112 @@ __global__ void __launch_bounds__(COPY_THREADS) copy_tables_kernel(const uint4* 
   }
 }
 
+// AdamW over many tensors in one launch (the non-matrix parameters that
+// train beside Muon: biases, norms, embeddings, the output layer).  Block b
+// handles chunk b of the concatenated tensors: it finds its tensor by binary
+// search in the chunk offsets, then each thread updates 4 consecutive
+// elements per pass in fp32 -- m = b1 m + (1-b1) g, v = b2 v + (1-b2) g^2,
+// p = (1 - lr wd) p - lr (m / bc1) / (sqrt(v / bc2) + eps) with bc = 1 - b^t
+// -- and writes p back with one rounding to its dtype.  22 bytes per bf16
+// element (p rw 4, g 2, m rw 8, v rw 8), 32 per fp32 element: HBM-bound.
+constexpr int ADAM_THREADS = 256;
+constexpr int ADAM_CHUNK = ADAM_THREADS * 4 * 4;  // 4 passes of 4 elements per thread
+
+// Every rounding is explicit (no contraction left to the compiler), so the
+// vector and element-by-element paths give the same bits.
+__device__ __forceinline__ void adam_elem(float& p, float g, float& m, float& v, const AdamwArgs& a) {
+  m = __fmaf_rn(a.beta1, m, __fmul_rn(a.omb1, g));
+  v = __fmaf_rn(a.beta2, v, __fmul_rn(__fmul_rn(a.omb2, g), g));
+  const float denom = __fadd_rn(__fsqrt_rn(__fdiv_rn(v, a.bc2)), a.eps);
+  p = __fmaf_rn(p, a.decay, -__fmul_rn(a.lr, __fdiv_rn(__fdiv_rn(m, a.bc1), denom)));
+}
+
+__global__ void __launch_bounds__(ADAM_THREADS) adamw_kernel(const AdamwArgs a) {
+  const long long chunk = blockIdx.x;
+  int lo = 0, hi = a.count - 1;  // last tensor whose first chunk <= chunk
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.chunk_start[mid] <= chunk) lo = mid;
+    else hi = mid - 1;
+  }
+  const int t = lo;
+  const long long n = a.numel[t];
+  const long long base = (chunk - a.chunk_start[t]) * ADAM_CHUNK;
+  float* M = a.M[t];
+  float* V = a.V[t];
+  const bool vec = a.aligned != 0;
+#pragma unroll 1
+  for (int pass = 0; pass < 4; ++pass) {
+    const long long e = base + (static_cast<long long>(pass) * ADAM_THREADS + threadIdx.x) * 4;
+    if (e >= n) break;
+    if (vec && e + 4 <= n) {
+      float4 m4 = *reinterpret_cast<const float4*>(M + e);
+      float4 v4 = *reinterpret_cast<const float4*>(V + e);
+      float pv[4], gv[4];
+      if (a.p_f32) {
+        const float4 p4 = *reinterpret_cast<const float4*>(static_cast<const float*>(a.P[t]) + e);
+        const float4 g4 = *reinterpret_cast<const float4*>(static_cast<const float*>(a.G[t]) + e);
+        pv[0] = p4.x; pv[1] = p4.y; pv[2] = p4.z; pv[3] = p4.w;
+        gv[0] = g4.x; gv[1] = g4.y; gv[2] = g4.z; gv[3] = g4.w;
+      } else {
+        const uint2 pu = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.P[t]) + e);
+        const uint2 gu = *reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(a.G[t]) + e);
+        const __nv_bfloat162* ph = reinterpret_cast<const __nv_bfloat162*>(&pu);
+        const __nv_bfloat162* gh = reinterpret_cast<const __nv_bfloat162*>(&gu);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const float2 pf = __bfloat1622float2(ph[q]), gf = __bfloat1622float2(gh[q]);
+          pv[2 * q] = pf.x; pv[2 * q + 1] = pf.y;
+          gv[2 * q] = gf.x; gv[2 * q + 1] = gf.y;
+        }
+      }
+      adam_elem(pv[0], gv[0], m4.x, v4.x, a);
+      adam_elem(pv[1], gv[1], m4.y, v4.y, a);
+      adam_elem(pv[2], gv[2], m4.z, v4.z, a);
+      adam_elem(pv[3], gv[3], m4.w, v4.w, a);
+      *reinterpret_cast<float4*>(M + e) = m4;
+      *reinterpret_cast<float4*>(V + e) = v4;
+      if (a.p_f32) {
+        *reinterpret_cast<float4*>(static_cast<float*>(a.P[t]) + e) = make_float4(pv[0], pv[1], pv[2], pv[3]);
+      } else {
+        uint2 pu;
+        __nv_bfloat162* ph = reinterpret_cast<__nv_bfloat162*>(&pu);
+        ph[0] = __floats2bfloat162_rn(pv[0], pv[1]);
+        ph[1] = __floats2bfloat162_rn(pv[2], pv[3]);
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.P[t]) + e) = pu;
+      }
+    } else {
+      for (int k = 0; k < 4 && e + k < n; ++k) {
+        const long long i = e + k;
+        float pv, gv;
+        if (a.p_f32) {
+          pv = static_cast<const float*>(a.P[t])[i];
+          gv = static_cast<const float*>(a.G[t])[i];
+        } else {
+          pv = __bfloat162float(static_cast<const __nv_bfloat16*>(a.P[t])[i]);
+          gv = __bfloat162float(static_cast<const __nv_bfloat16*>(a.G[t])[i]);
+        }
+        float m = M[i], v = V[i];
+        adam_elem(pv, gv, m, v, a);
+        M[i] = m;
+        V[i] = v;
+        if (a.p_f32) static_cast<float*>(a.P[t])[i] = pv;
+        else static_cast<__nv_bfloat16*>(a.P[t])[i] = __float2bfloat16_rn(pv);
+      }
+    }
+  }
+}
+
 }  // namespace
+
+long long adamw_chunks(long long numel) { return (numel + ADAM_CHUNK - 1) / ADAM_CHUNK; }
+
+cudaError_t launch_adamw(const AdamwArgs& a, long long total_chunks, cudaStream_t st) {
+  if (a.count <= 0 || total_chunks <= 0) return cudaSuccess;
+  if (total_chunks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  adamw_kernel<<<static_cast<unsigned>(total_chunks), ADAM_THREADS, 0, st>>>(a);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_copy_tables(const void* const* src, void* const* dst, long long bytes, int cnt, int num_sms,
                                cudaStream_t st) {

@@ -23,8 +23,10 @@ def test_tensor_list_matches_plain_list():
 
 
 def test_marshalling_rejects_non_matrices():
-    with pytest.raises(ValueError):
-        B.TensorList([torch.empty(4, 4), torch.empty(2, 3, 4)])
+    tl = B.TensorList([torch.empty(4, 4), torch.empty(2, 3, 4)])   # fine for AdamW (any rank) ...
+    assert tl.shapes is None and len(tl) == 2
+    with pytest.raises(ValueError):                                 # ... but not as Muon matrices
+        B._shapes(tl)
     with pytest.raises(ValueError):
         B._shapes([torch.empty(8, 8).t()[:, :4]])
 
