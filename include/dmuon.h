@@ -128,7 +128,8 @@ int dmuon_step_ex(void* const* params, const void* const* grads, void* const* mo
  * compute stream.  Matrices of at most 256 KB whose host buffers are pinned
  * and 16-byte aligned are copied by a kernel that reads and writes the
  * mapped host memory, one launch per chunk; other matrices take one
- * copy-engine transfer each (DMUON_IO_COPY=dma|kernel forces one kind).
+ * copy-engine transfer each (DMUON_IO_COPY=dma|kernel forces one kind;
+ * out-kernel takes the kernel for every copy-out).
  *   params[i]          device, updated in place (as dmuon_step).
  *   grads_host[i]      host, rows_i x cols_i row-major; pinned (page-locked)
  *                      memory for the copies to run asynchronously.

@@ -762,13 +762,14 @@ size_t io_stride(long long rows, long long cols, bool g_f32) {
 // beside them (2 MB matrices: 4.0 ms against 6.0 ms).  "auto" takes the
 // kernel for groups of small matrices whose host buffers allow it.
 // DMUON_IO_COPY overrides.
-enum IoCopy { IO_AUTO = 0, IO_DMA = 1, IO_KERNEL = 2 };
+enum IoCopy { IO_AUTO = 0, IO_DMA = 1, IO_KERNEL = 2, IO_OUT_KERNEL = 3 };
 constexpr long long kIoKernelMaxBytes = 256 << 10;
 IoCopy io_copy_mode() {
   static const IoCopy v = [] {
     const char* e = getenv("DMUON_IO_COPY");
     if (e && strcmp(e, "dma") == 0) return IO_DMA;
     if (e && strcmp(e, "kernel") == 0) return IO_KERNEL;
+    if (e && strcmp(e, "out-kernel") == 0) return IO_OUT_KERNEL;
     return IO_AUTO;
   }();
   return v;
@@ -928,7 +929,7 @@ int run_step(Request& r) {
   // chunk (chunks alternate between the two slots in issue order).
   uint8_t* ws = static_cast<uint8_t*>(c.ws);
   std::vector<void*> host(ntab * static_cast<size_t>(r.count));
-  std::vector<char> kcopy(groups.size(), 0);  // host I/O through copy_tables_kernel
+  std::vector<char> kin(groups.size(), 0), kout(groups.size(), 0);  // host I/O through copy_tables_kernel
   std::vector<int> gstart(groups.size());
   {
     int pos = 0;
@@ -942,22 +943,26 @@ int run_step(Request& r) {
         ++pos;
       }
     }
-    if (r.grads_host && io_copy_mode() != IO_DMA) {
+    const IoCopy mode = io_copy_mode();
+    if (r.grads_host && mode != IO_DMA) {
       for (size_t k = 0; k < groups.size(); ++k) {
         const Group& gr = groups[k];
         const long long gbytes = gr.rows * gr.cols * (g_f32 ? 4 : 2);
         const long long wbytes = gr.rows * gr.cols * (f32 ? 4 : 2);
-        bool ok = gbytes % 16 == 0 && wbytes % 16 == 0 &&
-                  (io_copy_mode() == IO_KERNEL || std::max(gbytes, wbytes) <= kIoKernelMaxBytes);
-        for (size_t q = 0; q < gr.idx.size() && ok; ++q) {
+        const bool small = std::max(gbytes, wbytes) <= kIoKernelMaxBytes;
+        bool ok_in = gbytes % 16 == 0 && (mode == IO_KERNEL || small);
+        bool ok_out = r.params_host && wbytes % 16 == 0 && (mode != IO_AUTO || small);
+        for (size_t q = 0; q < gr.idx.size() && (ok_in || ok_out); ++q) {
           const int i = gr.idx[q];
-          void* hs = mapped_host(r.grads[i]);
-          void* hd = r.params_host ? mapped_host(r.params_host[i]) : nullptr;
-          ok = hs && aligned16(hs) && (!r.params_host || (hd && aligned16(hd) && aligned16(r.params[i])));
+          void* hs = ok_in ? mapped_host(r.grads[i]) : nullptr;
+          void* hd = ok_out ? mapped_host(r.params_host[i]) : nullptr;
+          ok_in = ok_in && hs && aligned16(hs);
+          ok_out = ok_out && hd && aligned16(hd) && aligned16(r.params[i]);
           host[4 * r.count + gstart[k] + q] = hs;
           host[5 * r.count + gstart[k] + q] = hd;
         }
-        kcopy[k] = ok ? 1 : 0;
+        kin[k] = ok_in ? 1 : 0;
+        kout[k] = ok_out ? 1 : 0;
       }
     }
     if (r.grads_host) {
@@ -1021,7 +1026,7 @@ int run_step(Request& r) {
         // chunk io_slots back has consumed that slot
         if (io_j >= io_slots) CUDA_TRY(cudaStreamWaitEvent(c.cin, c.g_free[slot], 0));
         const size_t bytes = static_cast<size_t>(g.rows) * g.cols * (g_f32 ? 4 : 2);
-        if (kcopy[k]) {
+        if (kin[k]) {
           CUDA_TRY(launch_k(KIND_OTHER, 0.0, 0.0, c.cin, [&] {
             return launch_copy_tables(dtab + 4 * r.count + p, dtab + p, static_cast<long long>(bytes), ch.cnt,
                                       c.num_sms, c.cin);
@@ -1053,7 +1058,7 @@ int run_step(Request& r) {
           CUDA_TRY(cudaEventRecord(c.w_done[slot], gs));
           CUDA_TRY(cudaStreamWaitEvent(c.cout, c.w_done[slot], 0));
           const size_t bytes = static_cast<size_t>(g.rows) * g.cols * (f32 ? 4 : 2);
-          if (kcopy[k]) {
+          if (kout[k]) {
             CUDA_TRY(launch_k(KIND_OTHER, 0.0, 0.0, c.cout, [&] {
               return launch_copy_tables(dtab + 2 * r.count + p, dtab + 5 * r.count + p,
                                         static_cast<long long>(bytes), ch.cnt, c.num_sms, c.cout);
