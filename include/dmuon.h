@@ -219,8 +219,11 @@ int dmuon_cache_entry(int i, char* buf, size_t len);
  */
 int dmuon_set_workspace(void* dev_ptr, size_t bytes);
 
-/* Scratch bytes the library would need for this set of shapes (planning
- * only, no allocation, no launch). */
+/* Scratch bytes the library would need for dmuon_step / dmuon_step_ex /
+ * dmuon_compute_update on this set of shapes (planning only, no allocation,
+ * no launch).  dmuon_step_host_io needs more (staging slots and a second
+ * compute region); with a caller workspace too small for the second region
+ * it runs its chunks on one stream. */
 int dmuon_workspace_size(const int64_t* shapes, int count, int param_dtype, size_t* bytes);
 
 /*

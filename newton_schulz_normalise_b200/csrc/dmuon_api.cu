@@ -373,7 +373,7 @@ Epilogue store_epi(void* D, long long ldd, long long sd, bool f32, float alpha, 
 }
 
 // Runs K1 (momentum + norm partials) and the finalize for a chunk.
-int run_momentum(DeviceCtx& c, const Chunk& ch, bool f32, bool g_f32, const Hyper& h, cudaStream_t s) {
+int run_momentum(const Chunk& ch, bool f32, bool g_f32, const Hyper& h, cudaStream_t s) {
   const Geo& g = *ch.g;
   MomentumArgs a{};
   a.G = ch.Gt;
@@ -926,7 +926,7 @@ int run_step(Request& r) {
 
   // pointer tables, grouped: for group k, its matrices are contiguous.  With
   // host gradients the G entries point at the staging slot of the matrix's
-  // chunk (chunks alternate between the two slots in issue order).
+  // chunk (chunks take the kIoSlots slots in turn, in issue order).
   uint8_t* ws = static_cast<uint8_t*>(c.ws);
   std::vector<void*> host(ntab * static_cast<size_t>(r.count));
   std::vector<char> kin(groups.size(), 0), kout(groups.size(), 0);  // host I/O through copy_tables_kernel
@@ -1038,7 +1038,7 @@ int run_step(Request& r) {
         CUDA_TRY(cudaEventRecord(c.g_ready[slot], c.cin));
         CUDA_TRY(cudaStreamWaitEvent(gs, c.g_ready[slot], 0));
       }
-      rc = run_momentum(c, ch, f32, g_f32, r.h, gs);
+      rc = run_momentum(ch, f32, g_f32, r.h, gs);
       if (rc) return rc;
       if (r.grads_host) CUDA_TRY(cudaEventRecord(c.g_free[slot], gs));
       if (miss[k] && c0 == 0) {
@@ -1269,7 +1269,7 @@ int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows,
   ch.Ot = reinterpret_cast<float* const*>(dtab + 3);
   ch.nblk = nblk;
   ch.aligned = aligned16(grad) && aligned16(momentum);
-  rc = run_momentum(c, ch, f32, o.grad_dtype == DMUON_F32, r.h, s);
+  rc = run_momentum(ch, f32, o.grad_dtype == DMUON_F32, r.h, s);
   if (rc) return rc;
   Epilogue fin{};
   fin.mode = EPI_OUT;

@@ -428,9 +428,27 @@ cudaError_t launch_wait_selftest(int* err, unsigned long long limit_ns, cudaStre
   return cudaGetLastError();
 }
 
+// Blocks of the momentum kernels resident on one SM (registers decide:
+// 64 per thread -> 4 blocks of 256), from the occupancy calculator.
+int momentum_blocks_per_sm() {
+  static int v = [] {
+    int a = 0, b = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&a, momentum_wide_kernel, EW_THREADS, 0) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, momentum_tall_kernel, EW_THREADS, 0) != cudaSuccess) {
+      cudaGetLastError();
+      return 4;
+    }
+    const int m = a < b ? a : b;
+    return m > 0 ? m : 4;
+  }();
+  return v;
+}
+
 int momentum_partials(int rows, int cols, int cnt, int num_sms) {
   const long long numel = static_cast<long long>(rows) * cols;
-  long long want = (8LL * num_sms + cnt - 1) / cnt;  // ~8 blocks (2048 threads) per SM over the group
+  // one resident wave over the group, rounded down (grid-stride loops take
+  // the rest): no second, partly empty wave
+  long long want = (static_cast<long long>(momentum_blocks_per_sm()) * num_sms) / cnt;
   long long cap;
   if (rows > cols)
     cap = static_cast<long long>((rows + TT - 1) / TT) * ((cols + TT - 1) / TT);

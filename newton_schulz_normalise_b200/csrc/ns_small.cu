@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(128, 2) ns_small_kernel(const SmallArgs p, int
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int r = tid;                    // TMEM lane = tile row of this thread
   const int j = r / p.mr, i = r % p.mr;  // matrix of the block, row inside it
   const int l = blockIdx.x * p.g + j;    // matrix index in the group
