@@ -6,7 +6,8 @@
 // same epilogue contract as the tensor-core GEMM.  32x32 output tile per
 // block of 256 threads (2x2 outputs each), 32-deep k slices staged in shared
 // memory: the fp32 workloads are single matrices of a few hundred rows, so
-// small tiles are what spreads a product over the SMs.
+// small tiles are what spreads a product over the SMs; when even those leave
+// SMs idle, K is split over a cluster of 2-8 CTAs (simt_gemm_splitk_kernel).
 #include "internal.h"
 
 namespace dmuon {
@@ -68,12 +69,118 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const float* __restrict_
   for (int i = 0; i < 2; ++i) epilogue_row<2>(epi, l, m0 + ty * 2 + i, col, acc[i], M, N);
 }
 
+// Split-K over a thread-block cluster.  The fp32 products are small (a few
+// hundred rows), so 32 x 32 output tiles give fewer blocks than SMs; here a
+// cluster of S CTAs shares one output tile, CTA r accumulating the r-th
+// slice of K with the loop above.  The partial tiles are summed through
+// distributed shared memory in a fixed CTA order (so the result does not
+// depend on timing), and CTA r applies the epilogue to rows r*32/S ..
+// (r+1)*32/S - 1 of the tile.
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+__global__ void __launch_bounds__(256) simt_gemm_splitk_kernel(const float* __restrict__ A, long long lda, long long sa,
+                                                               const float* __restrict__ B, long long ldb, long long sb,
+                                                               int b_kmajor, int M, int N, int K, int S, int ks,
+                                                               const Epilogue epi) {
+  __shared__ float As[TK][TM + 1];
+  __shared__ float Bs[TK][TN + 1];
+  __shared__ float part[TM][TN];
+  const int l = blockIdx.z;
+  const int r = static_cast<int>(cluster_rank());  // K slice of this CTA
+  const int m0 = blockIdx.y * TM, n0 = (blockIdx.x / S) * TN;
+  const int tid = threadIdx.x;
+  const int tx = tid % 16, ty = tid / 16;
+  const float* Ab = A + static_cast<long long>(l) * sa;
+  const float* Bb = B + static_cast<long long>(l) * sb;
+  const int k_lo = r * ks, k_hi = min(K, k_lo + ks);
+  float acc[2][2] = {};
+  for (int k0 = k_lo; k0 < k_hi; k0 += TK) {
+    for (int i = tid; i < TM * TK; i += 256) {
+      const int rr = i / TK, k = i % TK;
+      const int gr = m0 + rr, gk = k0 + k;
+      As[k][rr] = (gr < M && gk < k_hi) ? Ab[static_cast<long long>(gr) * lda + gk] : 0.f;
+    }
+    for (int i = tid; i < TN * TK; i += 256) {
+      int c, k;
+      if (b_kmajor) {
+        c = i / TK;
+        k = i % TK;
+      } else {
+        k = i / TN;
+        c = i % TN;
+      }
+      const int gc = n0 + c, gk = k0 + k;
+      float v = 0.f;
+      if (gc < N && gk < k_hi)
+        v = b_kmajor ? Bb[static_cast<long long>(gc) * ldb + gk] : Bb[static_cast<long long>(gk) * ldb + gc];
+      Bs[k][c] = v;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int k = 0; k < TK; ++k) {
+      const float a0 = As[k][ty * 2], a1 = As[k][ty * 2 + 1];
+      const float b0 = Bs[k][tx * 2], b1 = Bs[k][tx * 2 + 1];
+      acc[0][0] = fmaf(a0, b0, acc[0][0]);
+      acc[0][1] = fmaf(a0, b1, acc[0][1]);
+      acc[1][0] = fmaf(a1, b0, acc[1][0]);
+      acc[1][1] = fmaf(a1, b1, acc[1][1]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) part[ty * 2 + i][tx * 2 + j] = acc[i][j];
+  cluster_sync();  // every slice's partial tile is in its CTA's shared memory
+  const int rows = TM / S;  // rows of the tile this CTA finishes
+  const uint32_t base = smem_u32(&part[0][0]);
+  for (int e = tid; e < rows * TN; e += 256) {
+    const int rr = r * rows + e / TN, c = e % TN;
+    const uint32_t off = static_cast<uint32_t>((rr * TN + c) * sizeof(float));
+    float v[1] = {0.f};
+    for (int q = 0; q < S; ++q) v[0] += ld_dsmem_f32(mapa_shared(base + off, static_cast<uint32_t>(q)));
+    if (n0 + c < N) epilogue_row<1>(epi, l, m0 + rr, n0 + c, v, M, N);
+  }
+  cluster_sync();  // no CTA leaves while another still reads its partial tile
+}
+
 }  // namespace
 
 cudaError_t launch_simt_gemm(const SimtGemm& g, cudaStream_t s) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0 || g.batch <= 0) return cudaSuccess;
   if (g.batch > 65535) return cudaErrorInvalidValue;
-  dim3 grid((g.N + TN - 1) / TN, (g.M + TM - 1) / TM, g.batch);
+  const int tiles_n = (g.N + TN - 1) / TN, tiles_m = (g.M + TM - 1) / TM;
+  const long long tiles = static_cast<long long>(tiles_n) * tiles_m * g.batch;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  // split K over a cluster when the tiles alone leave SMs idle, keeping at
+  // least one TK-deep slice per CTA
+  int S = 1;
+  while (S < 8 && tiles * S < sms && g.K >= 2 * S * TK) S *= 2;
+  if (S > 1) {
+    const int ks = ((g.K + S * TK - 1) / (S * TK)) * TK;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles_n * S), static_cast<unsigned>(tiles_m), static_cast<unsigned>(g.batch));
+    cfg.blockDim = dim3(256);
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = static_cast<unsigned>(S);
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, simt_gemm_splitk_kernel, g.A, g.lda, g.sa, g.B, g.ldb, g.sb, g.b_kmajor ? 1 : 0,
+                              g.M, g.N, g.K, S, ks, g.epi);
+  }
+  dim3 grid(tiles_n, tiles_m, g.batch);
   simt_gemm_kernel<<<grid, 256, 0, s>>>(g.A, g.lda, g.sa, g.B, g.ldb, g.sb, g.b_kmajor ? 1 : 0, g.M, g.N, g.K,
                                         g.epi);
   return cudaGetLastError();
