@@ -160,10 +160,11 @@ cudaError_t launch_simt_gemm(const SimtGemm& g, cudaStream_t s) {
     cudaGetLastError();
     sms = 148;
   }
-  // split K over a cluster when the tiles alone leave SMs idle, keeping at
-  // least one TK-deep slice per CTA
+  // split K over a cluster until the grid covers two CTAs per SM (each CTA
+  // holds 12.5 KB of shared memory and 32 registers per thread, so several
+  // fit), keeping at least one TK-deep slice per CTA
   int S = 1;
-  while (S < 8 && tiles * S < sms && g.K >= 2 * S * TK) S *= 2;
+  while (S < 8 && tiles * S < 2 * sms && g.K >= 2 * S * TK) S *= 2;
   if (S > 1) {
     const int ks = ((g.K + S * TK - 1) / (S * TK)) * TK;
     cudaLaunchConfig_t cfg = {};
