@@ -841,7 +841,7 @@ int run_step(Request& r) {
         miss[k] = true;
       }
     }
-    const int nblk = momentum_partials(geos[k].rows, geos[k].cols, gr.chunk, c.num_sms);
+    const int nblk = momentum_partials(geos[k].rows, geos[k].cols);
     Layout L = make_layout(geos[k], gr.chunk, nblk);
     size_t need = L.total;
     if (miss[k]) need += 2 * align256(static_cast<size_t>(gr.chunk) * geos[k].x_elems() * geos[k].esz) + 256;
@@ -1008,7 +1008,7 @@ int run_step(Request& r) {
       ch.g = &g;
       ch.cnt = std::min(gr.chunk, total - c0);
       ch.base = ws + region_off[ln];
-      ch.nblk = momentum_partials(g.rows, g.cols, gr.chunk, c.num_sms);
+      ch.nblk = momentum_partials(g.rows, g.cols);
       ch.L = make_layout(g, gr.chunk, ch.nblk);
       const int p = gstart[k] + c0;
       ch.Gt = dtab + p;
@@ -1239,7 +1239,7 @@ int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows,
   int sms = 0;
   CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   const Geo g = make_geo(rows, cols, f32);
-  const int nblk = momentum_partials(g.rows, g.cols, 1, sms);
+  const int nblk = momentum_partials(g.rows, g.cols);
   const Layout L = make_layout(g, 1, nblk);
   const size_t header = 256;  // 4 pointer slots and the device error word
   const size_t need = header + L.total;
@@ -1545,7 +1545,7 @@ int dmuon_workspace_size(const int64_t* shapes, int count, int param_dtype, size
   for (auto& kv : counts) {
     Geo g = make_geo(kv.first.first, kv.first.second, f32);
     int ch = chunk_size(g, kv.second);
-    Layout L = make_layout(g, ch, momentum_partials(g.rows, g.cols, ch, sms));
+    Layout L = make_layout(g, ch, momentum_partials(g.rows, g.cols));
     const size_t n_tune = align256(L.total + 2 * align256(static_cast<size_t>(ch) * g.x_elems() * g.esz) + 256);
     need = std::max(need, n_tune);
     const bool maybe_small = !f32 && kv.second <= ch && (tc_gemm_tiles(g.m, g.n, ch, 128, false) < 2LL * sms ||

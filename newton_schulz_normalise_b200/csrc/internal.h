@@ -61,7 +61,7 @@ struct MomentumArgs {
 };
 cudaError_t launch_momentum(const MomentumArgs& a, cudaStream_t s);
 // Number of partial slots launch_momentum uses for this shape.
-int momentum_partials(int rows, int cols, int cnt, int num_sms);
+int momentum_partials(int rows, int cols);
 
 // s[l] = 1 / (sqrt(sum partials[l][:]) + eps),  s2[l] = s[l]^2.
 cudaError_t launch_norm_finalize(const float* partials, int nblk, int cnt, float eps, float* s, float* s2,
