@@ -232,7 +232,9 @@ def run_reference(args, w):
         "impl": "reference", "metric": METRIC, "value": val, "unit": "ms", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": val, "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "matrices": len(w.shapes())},
+        "config": {"workload": w.name, "matrices": len(w.shapes()),
+                   "shapes": sorted({f"{r}x{c}" for r, c in w.shapes()}), "ns_steps": w.ns_steps,
+                   "lr": w.lr, "wd": w.wd, "mu": w.mu, "parallelism": "fp64 oracle on rank 0's host cores"},
         "cpu_baseline": {"value": val, "unit": "ms", "cores": base["cores"], "kind": "oracle",
                          "sample": base["sample"]},
         "e2e": {"value": val, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
