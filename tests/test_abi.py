@@ -104,3 +104,38 @@ def test_set_workspace_alignment(dmuon_lib):
     L = dmuon_lib
     assert L.lib.dmuon_set_workspace(ctypes.c_void_p(0x1001), 4096) == L.DMUON_ERR_INVALID
     assert L.lib.dmuon_set_workspace(None, 0) == L.DMUON_OK
+
+
+def test_header_compiles_and_links_as_plain_c(dmuon_lib, tmp_path):
+    """A C99 program includes include/dmuon.h, links libdmuon.so and calls
+    entry points that need no GPU: the boundary is usable without C++ or
+    Python."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    src = tmp_path / "abi_check.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "dmuon.h"
+int main(void) {
+  dmuon_options o;
+  dmuon_options_init(&o);
+  if (dmuon_version() != 1 || o.variant != DMUON_VARIANT_AUTO || o.mom_dtype != DMUON_F32) return 1;
+  /* count 0 is a no-op; a null pointer array is rejected before any launch */
+  if (dmuon_step(NULL, NULL, NULL, NULL, 0, 0.02f, 0.1f, 0.95f, 5, NULL) != 0) return 2;
+  int64_t shape[2] = {4, 4};
+  int rc = dmuon_step(NULL, NULL, NULL, shape, 1, 0.02f, 0.1f, 0.95f, 5, NULL);
+  if (rc != DMUON_ERR_INVALID) return 3;
+  printf("%d %s\n", rc, dmuon_last_error());
+  return 0;
+}
+''')
+    lib = Path(dmuon_lib.LIB_PATH)
+    exe = tmp_path / "abi_check"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", f"-I{ROOT / 'include'}", str(src), "-o", str(exe),
+                    f"-L{lib.parent}", "-ldmuon", f"-Wl,-rpath,{lib.parent}"], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert r.stdout.startswith(str(dmuon_lib.DMUON_ERR_INVALID))
