@@ -5,15 +5,17 @@
 
 A step is one call of the library's ``dmuon_step`` over a whole parameter set
 (momentum, normalisation, 5 quintic Newton-Schulz steps, scale, decay and the
-parameter write for every matrix).  Default workload: 64 square 1024 x 1024
-bf16 weights with fp32 momenta (grads ~ N(0, 1e-3^2)).  Inputs are resident
-in HBM before the timed region; they total 537 MB (> 126 MB of L2), so no L2
+parameter write for every matrix).  Default workload: the matrix set of a
+Llama-style 8B model (32 layers of q 4096^2, k and v 4096 x 1024, o 4096^2,
+gate and up 4096 x 14336, down 14336 x 4096; 224 matrices, 6.98 G elements),
+bf16 weights and grads ~ N(0, 1e-3^2), fp32 momenta.  Inputs are resident in
+HBM before the timed region; they total 56 GB (> 126 MB of L2), so no L2
 flush is needed between steps.
 
 Prints one JSON line (rank 0).  N > 1 runs independent replicas, one per
 rank (the step has no exchange on one parameter set); timing is the max over
 ranks of the device-timed region.  ``--impl reference`` times the fp64 CPU
-oracle on a bounded sample of the same workload instead.
+oracle on bounded samples of the same workload instead.
 """
 from __future__ import annotations
 
@@ -32,6 +34,7 @@ ROOT = Path(__file__).resolve().parent
 sys.path.insert(0, str(ROOT))
 
 METRIC = "Muon step ms per param set; NS TFLOPS as % of B200 bf16 dense peak"
+DEFAULT_WORKLOAD = "llama8b-matrices-bf16"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 10 ** 6
 # fp32 FFMA peak from unit counts and clock: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz
@@ -122,45 +125,74 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU baseline (oracle)
-def cpu_baseline(w, budget_s=12.0):
-    """The fp64 oracle as it stands, on the first matrices of the workload,
-    as many as fit in ~budget_s, extrapolated to the whole parameter set."""
-    import numpy as np
-    import torch
-    import oracle.muon_oracle as ora
-    from newton_schulz_normalise_b200 import workloads as wl
+# A parameter set whose direct-form Newton-Schulz work is at most this many
+# FLOPs is timed in full by the fp64 oracle (the fp32 256 x 512 set and the
+# 64 x 1024^2 set: a few seconds on a many-core host).  Larger sets time one
+# matrix of every distinct shape and scale each by its count ("extrapolated").
+FULL_ORACLE_FLOPS = 4.0e12
 
+
+def oracle_sample(w):
+    """Matrix indices the oracle times and whether they are the whole set."""
     shapes = w.shapes()
+    if sum(ns_flops(r, c, w.ns_steps, "direct") for r, c in shapes) <= FULL_ORACLE_FLOPS:
+        return list(range(len(shapes))), False
+    first = {}
+    for i, s in enumerate(shapes):
+        first.setdefault(s, i)
+    return sorted(first.values()), True
+
+
+def oracle_inputs(w, indices):
+    """fp64 host copies of (W, G, M) for the given matrices (CPU generator:
+    same shapes and distributions as the device draw; values do not affect
+    the oracle's time)."""
+    from newton_schulz_normalise_b200 import workloads as wl
+    Ws, Gs, Ms = wl.generate(w, device="cpu", indices=indices)
+    return [(a.double().numpy(), b.double().numpy(), c.double().numpy()) for a, b, c in zip(Ws, Gs, Ms)]
+
+
+def oracle_seconds(w, inp):
+    """Wall time of oracle.muon_step (as it stands) on one matrix."""
+    import oracle.muon_oracle as ora
+    W, G, M = inp
+    t0 = time.perf_counter()
+    ora.muon_step(W, G, M, w.lr, w.wd, w.mu, w.ns_steps)
+    return time.perf_counter() - t0
+
+
+def oracle_set_ms(w, per_shape_s):
+    """ms per parameter set from mean seconds per matrix of each shape."""
+    return 1e3 * sum(statistics.mean(per_shape_s[s]) for s in w.shapes())
+
+
+def _threads():
+    import torch
     cores = len(os.sched_getaffinity(0))
     torch.set_num_threads(cores)
-    done, spent = 0, 0.0
+    return cores
+
+
+def cpu_baseline(w):
+    """The fp64 oracle as it stands on the host cores: the whole parameter set
+    when it is small (FULL_ORACLE_FLOPS), else one matrix of every distinct
+    shape, each scaled by its count."""
+    cores = _threads()
+    idx, extrapolated = oracle_sample(w)
+    shapes = w.shapes()
+    inputs = oracle_inputs(w, idx)
     per_shape = {}
-    for i, (r, c) in enumerate(shapes):
-        if (r, c) in per_shape and len(per_shape[(r, c)]) >= 2:
-            continue
-        Ws, Gs, Ms = wl.generate(w, device="cpu", indices=[i])
-        W = Ws[0].double().numpy()
-        G = Gs[0].double().numpy()
-        M = Ms[0].double().numpy()
-        t0 = time.perf_counter()
-        ora.muon_step(W, G, M, w.lr, w.wd, w.mu, w.ns_steps)
-        dt = time.perf_counter() - t0
-        per_shape.setdefault((r, c), []).append(dt)
-        done += 1
-        spent += dt
-        if spent > budget_s:
-            break
-    total_s = 0.0
-    for (r, c) in shapes:
-        ts = per_shape.get((r, c))
-        if ts is None:  # not reached within budget: scale by flops from a timed shape
-            (r0, c0), t0s = next(iter(per_shape.items()))
-            ts = [statistics.mean(t0s) * ns_flops(r, c, 5, "direct") / ns_flops(r0, c0, 5, "direct")]
-        total_s += statistics.mean(ts)
+    for i, inp in zip(idx, inputs):
+        per_shape.setdefault(shapes[i], []).append(oracle_seconds(w, inp))
+    val = oracle_set_ms(w, per_shape)
+    how = ("one matrix of each of the %d shapes, scaled by its count" % len(per_shape) if extrapolated
+           else "the whole set")
     return {
-        "value": total_s * 1e3, "unit": "ms", "cores": cores, "kind": "oracle",
-        "sample": f"{done} of {len(shapes)} matrices timed one by one (fp64 numpy, BLAS on "
-                  f"{cores} threads), mean per shape x count",
+        "value": val, "unit": "ms", "cores": cores, "kind": "oracle",
+        "sample": f"{len(idx)} of {len(shapes)} matrices timed one by one ({how}); fp64 numpy, "
+                  f"BLAS on {cores} threads",
+        "extrapolated": extrapolated, "matrices_timed": len(idx),
+        "per_shape_ms": {f"{r}x{c}": round(1e3 * statistics.mean(t), 3) for (r, c), t in per_shape.items()},
         "cpu": _cpu_model(),
         "adamw": adamw_oracle_time(),
     }
@@ -218,42 +250,81 @@ def job_value(ms_max, steps, world_size):
 
 
 def run_reference(args, w):
+    """The oracle arm.  A step times one bounded sample: the whole parameter
+    set when it is small, else one matrix, taking the distinct shapes in turn.
+    ms_per_step is the mean time of the timed samples as they ran; value is
+    the ms per parameter set they imply (scaled by each shape's count when the
+    samples are single matrices, and then marked extrapolated)."""
     ws, rank, _ = dist_env()
     if rank != 0:
         return 0
-    times = []
-    base = None
-    for _ in range(args.warmup + args.steps):
-        # each step times at least one matrix; the whole run stays near 2 minutes
-        base = cpu_baseline(w, budget_s=max(0.3, 120.0 / max(args.steps + args.warmup, 1)))
-        times.append(base["value"])
-    val = statistics.mean(times[args.warmup:]) if len(times) > args.warmup else times[-1]
+    cores = _threads()
+    idx, extrapolated = oracle_sample(w)
+    shapes = w.shapes()
+    inputs = oracle_inputs(w, idx)
+    per_shape, step_s = {}, []
+    t_run0 = time.perf_counter()
+    for k in range(args.warmup + args.steps):
+        if extrapolated:
+            j = k % len(idx)
+            dt = oracle_seconds(w, inputs[j])
+            if k >= args.warmup or len(idx) > args.steps:
+                per_shape.setdefault(shapes[idx[j]], []).append(dt)
+        else:
+            dt = 0.0
+            for i, inp in zip(idx, inputs):
+                t = oracle_seconds(w, inp)
+                dt += t
+                if k >= args.warmup:
+                    per_shape.setdefault(shapes[i], []).append(t)
+        if k >= args.warmup:
+            step_s.append(dt)
+    for i, inp in zip(idx, inputs):  # a run too short to meet every shape: time the rest once
+        if shapes[i] not in per_shape:
+            per_shape[shapes[i]] = [oracle_seconds(w, inp)]
+    run_s = time.perf_counter() - t_run0
+    val = oracle_set_ms(w, per_shape)
+    sample = (f"step k times matrix {{{', '.join(str(i) for i in idx)}}}[k mod {len(idx)}] (one of each shape); "
+              f"value = sum over shapes of count x mean time" if extrapolated
+              else f"every step times all {len(shapes)} matrices one by one")
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": "ms", "n_gpus": ws,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": val, "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "matrices": len(w.shapes()),
-                   "shapes": sorted({f"{r}x{c}" for r, c in w.shapes()}), "ns_steps": w.ns_steps,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.mean(step_s) if step_s else None,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "matrices": len(shapes),
+                   "shapes": sorted({f"{r}x{c}" for r, c in shapes}), "ns_steps": w.ns_steps,
                    "lr": w.lr, "wd": w.wd, "mu": w.mu, "parallelism": "fp64 oracle on rank 0's host cores"},
-        "cpu_baseline": {"value": val, "unit": "ms", "cores": base["cores"], "kind": "oracle",
-                         "sample": base["sample"]},
+        "extrapolated": extrapolated,
+        "cpu_baseline": {"value": val, "unit": "ms", "cores": cores, "kind": "oracle", "sample": sample,
+                         "extrapolated": extrapolated,
+                         "per_shape_ms": {f"{r}x{c}": round(1e3 * statistics.mean(t), 3)
+                                          for (r, c), t in per_shape.items()},
+                         "run_s": round(run_s, 2)},
         "e2e": {"value": val, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
 
 
-def profile_traffic(kernel_file: Path):
+# ncu summaries of the CTA-pair GEMM per bench workload; each holds the
+# per-launch DRAM traffic of the bench's launches and the hash of the kernel
+# source it was taken on.
+PAIR_PROFILES = {"batch64-1024x1024-bf16": "tc_gemm_pair_batch64-1024x1024.md",
+                 "llama8b-matrices-bf16": "tc_gemm_pair_llama8b-matrices.md"}
+
+
+def profile_traffic(kernel_file: Path, workload: str):
     """Per-launch DRAM traffic of the dominant kernel from the committed ncu
-    summary, if it was taken on the current kernel source."""
+    summary of this workload, if it was taken on the current kernel source."""
     import hashlib
-    summ = ROOT / "profiles" / "tc_gemm_pair_batch64-1024x1024.md"
-    if not summ.exists():
+    name = PAIR_PROFILES.get(workload)
+    summ = ROOT / "profiles" / name if name else None
+    if summ is None or not summ.exists():
         return None
     sha = hashlib.sha256(kernel_file.read_bytes()).hexdigest()[:16]
-    txt = summ.read_text()
     src, traffic = None, None
-    for line in txt.splitlines():
+    for line in summ.read_text().splitlines():
         if line.startswith("kernel_source_sha256_16:"):
             src = line.split(":", 1)[1].strip()
         if line.startswith("traffic_bytes_per_launch:"):
@@ -293,9 +364,9 @@ def adamw_measure(dev, stream, torch_dtype, iters=20):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="batch64-1024x1024-bf16")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cache-file", default=None,
@@ -389,15 +460,19 @@ def main():
     clocks.stop()
     clk = clocks.summary(t_host0, t_host1)
 
-    # ---------------- per-kernel timing pass (same steps, events around each launch)
+    # ---------------- per-kernel timing pass: the same steps again, the
+    # Newton-Schulz products of every chunk bracketed by one pair of events
+    # (no event between two products), other launches by their own pair;
+    # about 3 s of steps
     B.dmuon_timing_reset()
     B.dmuon_timing_enable(True)
-    kt_steps = min(args.steps, 50)
+    kt_steps = max(1, min(args.steps, 50, int(3000.0 / max(ms / args.steps, 1e-3))))
     for _ in range(kt_steps):
         step()
     torch.cuda.synchronize()
     B.dmuon_timing_enable(False)
-    kinds = {k: B.dmuon_timing_get(k) for k in (B.KIND_TC_GEMM, B.KIND_EW, B.KIND_SIMT_GEMM, B.KIND_OTHER)}
+    kinds = {k: B.dmuon_timing_get(k) for k in (B.KIND_TC_GEMM, B.KIND_EW, B.KIND_SIMT_GEMM, B.KIND_OTHER,
+                                                 B.KIND_TC_GEMM_PAIR)}
     B.dmuon_timing_reset()
 
     # ---------------- end to end through the C ABI with host buffers
@@ -445,37 +520,53 @@ def main():
         f = e.split()
         variants[(int(f[0]), int(f[1]))] = f[4]
     gemm = kinds[B.KIND_TC_GEMM]
+    pairk = kinds[B.KIND_TC_GEMM_PAIR]
     simt = kinds[B.KIND_SIMT_GEMM]
     # executed NS FLOPs per step (symmetric products count their computed tiles only)
     flops = (gemm["flops"] + simt["flops"]) / kt_steps
     dense = sum(ns_flops(r, c, w.ns_steps, variants.get((r, c), "direct")) for r, c in shapes)
     tflops = flops / (ms_per_step * 1e-3) / 1e12
     peak_tc = peaks["bf16_tflops"]
-    ach = gemm["flops"] / (gemm["ms"] * 1e-3) / 1e12 if gemm["ms"] > 0 else 0.0
-    # the committed ncu summary covers the pair kernel on the default workload only
-    traffic = (profile_traffic(ROOT / "newton_schulz_normalise_b200" / "csrc" / "gemm_tc.cu")
-               if w.name == "batch64-1024x1024-bf16" else None)
-    tiles = {e.split()[5] for e in plans}
+    peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     variants_used = {e.split()[4] for e in plans}
-    gemm_kernel = "tc_gemm2_kernel (CTA pair)" if tiles == {"512"} else "tc_gemm_kernel / tc_gemm2_kernel"
-    if variants_used == {"batched"}:
-        gemm_kernel = "ns_small_kernel (resident)"
-    if gemm["launches"] > 0:
-        roofline = {"bound": "tensor", "kernel": gemm_kernel, "achieved": round(ach, 1),
+    # the dominant kernel: the CTA-pair GEMM when its chains hold most of the
+    # tensor-core time, else the tensor-core GEMMs together (one-CTA tiles,
+    # resident kernel), else the fp32 SIMT GEMM
+    if pairk["launches"] > 0 and pairk["ms"] >= 0.5 * gemm["ms"]:
+        dom, dom_kernel, prof = pairk, "tc_gemm2_kernel (CTA pair)", "pair"
+    elif gemm["launches"] > 0:
+        dom, prof = gemm, None
+        dom_kernel = ("ns_small_kernel (resident)" if variants_used == {"batched"}
+                      else "tc_gemm_kernel / tc_gemm2_kernel / ns_small_kernel")
+    else:
+        dom, dom_kernel, prof = simt, "simt_gemm_kernel (fp32 FFMA)", None
+    ach = dom["flops"] / (dom["ms"] * 1e-3) / 1e12 if dom["ms"] > 0 else 0.0
+    share = round(dom["ms"] / kt_steps / ms_per_step, 3) if ms_per_step else None
+    per_launch_ms = dom["ms"] / dom["launches"] if dom["launches"] else None
+    if dom is not simt:
+        traffic = (profile_traffic(ROOT / "newton_schulz_normalise_b200" / "csrc" / "gemm_tc.cu", w.name)
+                   if prof == "pair" else None)
+        roofline = {"bound": "tensor", "kernel": dom_kernel, "achieved": round(ach, 1),
                     "peak": peak_tc, "unit": "TFLOP/s", "frac": round(ach / peak_tc, 4),
                     "traffic": traffic, "peak_source": f"{peaks['_source']} bf16_tflops (burst)",
-                    "frac_of_sustained": round(ach / peaks.get("bf16_tflops_sustained",
-                                                               FALLBACK_PEAKS["bf16_tflops_sustained"]), 4),
-                    "launches": gemm["launches"] // kt_steps,
-                    "share_of_step": round(gemm["ms"] / kt_steps / ms_per_step, 3) if ms_per_step else None}
+                    "frac_of_sustained": round(ach / peak_sus, 4),
+                    "launches": dom["launches"] // kt_steps,
+                    "ms_per_launch": round(per_launch_ms, 4) if per_launch_ms else None,
+                    "flops_per_launch": dom["flops"] / dom["launches"] if dom["launches"] else None,
+                    "share_of_step": share}
+        if dom is pairk:  # all tensor-core GEMMs together, for reference
+            roofline["all_tc_gemms"] = {
+                "achieved": round(gemm["flops"] / (gemm["ms"] * 1e-3) / 1e12, 1) if gemm["ms"] > 0 else 0.0,
+                "launches": gemm["launches"] // kt_steps,
+                "share_of_step": round(gemm["ms"] / kt_steps / ms_per_step, 3) if ms_per_step else None}
     else:  # fp32 path: Newton-Schulz on the CUDA cores (FFMA)
-        ach_s = simt["flops"] / (simt["ms"] * 1e-3) / 1e12 if simt["ms"] > 0 else 0.0
-        roofline = {"bound": "alu", "kernel": "simt_gemm_kernel (fp32 FFMA)", "achieved": round(ach_s, 2),
-                    "peak": round(FP32_FFMA_TFLOPS, 1), "unit": "TFLOP/s", "frac": round(ach_s / FP32_FFMA_TFLOPS, 4),
+        roofline = {"bound": "alu", "kernel": dom_kernel, "achieved": round(ach, 2),
+                    "peak": round(FP32_FFMA_TFLOPS, 1), "unit": "TFLOP/s", "frac": round(ach / FP32_FFMA_TFLOPS, 4),
                     "traffic": None,
                     "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz",
-                    "launches": simt["launches"] // kt_steps,
-                    "share_of_step": round(simt["ms"] / kt_steps / ms_per_step, 3) if ms_per_step else None}
+                    "launches": dom["launches"] // kt_steps,
+                    "ms_per_launch": round(per_launch_ms, 4) if per_launch_ms else None,
+                    "share_of_step": share}
     ew = kinds[B.KIND_EW]
     ew_gbs = ew["bytes"] / (ew["ms"] * 1e-3) / 1e9 if ew["ms"] > 0 else 0.0
 

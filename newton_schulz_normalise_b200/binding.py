@@ -24,7 +24,7 @@ DMUON_BF16 = 0
 DMUON_F32 = 1
 
 VARIANTS = {"auto": 0, "direct": 1, "gram": 2, "batched": 3}
-KIND_TC_GEMM, KIND_EW, KIND_SIMT_GEMM, KIND_OTHER = 0, 1, 2, 3
+KIND_TC_GEMM, KIND_EW, KIND_SIMT_GEMM, KIND_OTHER, KIND_TC_GEMM_PAIR = 0, 1, 2, 3, 4
 
 # every entry point include/dmuon.h declares
 EXPORTS = (

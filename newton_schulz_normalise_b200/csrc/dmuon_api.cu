@@ -60,16 +60,26 @@ bool trace_on() {
 }
 
 // ------------------------------------------------------------------ timing
+// While timing is enabled, a launch outside a TimedChain is bracketed by its
+// own pair of events.  A TimedChain (the Newton-Schulz products of one chunk,
+// run_ns) is bracketed by ONE pair of events around all of its launches:
+// nothing else is enqueued between them, so the window is the chain's device
+// time, with no event between two of its kernels to delay the next launch or
+// break programmatic dependent launch.  A record's kind is that of its first
+// launch; `pair` marks chains of the CTA-pair GEMM.
 struct TimedLaunch {
   int kind;
+  bool pair;
   cudaEvent_t a, b;
   double flops, bytes;
+  long long launches;
 };
 std::mutex g_tmu;
 std::atomic<int> g_timing{0};
 std::vector<TimedLaunch> g_timed;
 std::vector<cudaEvent_t> g_event_pool;
 std::atomic<long long> g_launches{0};
+thread_local TimedLaunch* t_chain = nullptr;
 
 cudaEvent_t take_event() {
   if (!g_event_pool.empty()) {
@@ -83,19 +93,60 @@ cudaEvent_t take_event() {
 }
 
 // Runs `launch` (which enqueues one kernel on `s`), bracketed by events when
-// timing is enabled.
+// timing is enabled and no chain is open.
 template <class F>
 cudaError_t launch_k(int kind, double flops, double bytes, cudaStream_t s, F&& launch) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (!g_timing.load(std::memory_order_relaxed)) return launch();
+  if (t_chain) {
+    if (t_chain->launches == 0) t_chain->kind = kind;
+    t_chain->flops += flops;
+    t_chain->bytes += bytes;
+    ++t_chain->launches;
+    return launch();
+  }
   std::lock_guard<std::mutex> lk(g_tmu);
-  TimedLaunch t{kind, take_event(), take_event(), flops, bytes};
+  TimedLaunch t{kind, false, take_event(), take_event(), flops, bytes, 1};
   cudaEventRecord(t.a, s);
   cudaError_t e = launch();
   cudaEventRecord(t.b, s);
   g_timed.push_back(t);
   return e;
 }
+
+// Scope of one timed chain of launches on stream `s` (no-op unless timing).
+class TimedChain {
+ public:
+  TimedChain(cudaStream_t s, bool pair) : s_(s) {
+    if (!g_timing.load(std::memory_order_relaxed) || t_chain) return;
+    {
+      std::lock_guard<std::mutex> lk(g_tmu);
+      rec_ = TimedLaunch{KIND_OTHER, pair, take_event(), take_event(), 0.0, 0.0, 0};
+    }
+    cudaEventRecord(rec_.a, s_);
+    t_chain = &rec_;
+    on_ = true;
+  }
+  ~TimedChain() {
+    if (!on_) return;
+    t_chain = nullptr;
+    cudaEventRecord(rec_.b, s_);
+    std::lock_guard<std::mutex> lk(g_tmu);
+    if (rec_.launches > 0) {
+      g_timed.push_back(rec_);
+    } else {
+      g_event_pool.push_back(rec_.a);
+      g_event_pool.push_back(rec_.b);
+    }
+  }
+  TimedChain(const TimedChain&) = delete;
+  TimedChain& operator=(const TimedChain&) = delete;
+
+ private:
+  cudaStream_t s_;
+  TimedLaunch rec_{};
+  bool on_ = false;
+};
 
 // ------------------------------------------------------------------ device context
 struct DeviceCtx {
@@ -403,7 +454,8 @@ int run_momentum(const Chunk& ch, bool f32, bool g_f32, const Hyper& h, cudaStre
 }
 
 // Newton-Schulz on X0 (unnormalised U, scale s folded into the first
-// products), finishing with `fin` (apply / out / store) on the result.
+// products), finishing with `fin` (apply / out / store) on the result.  Its
+// launches are timed as one chain.
 int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const Hyper& h, const Epilogue& fin_in,
            int cnt, cudaStream_t s) {
   const Geo& g = *ch.g;
@@ -421,6 +473,7 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
     fin.C = nullptr;
     cudaError_t e = launch_k(KIND_OTHER, 0.0, 0.0, s, [&] {
       return launch_scale_epilogue(X0, g.ldx, f32, m, n, cnt, sv, fin, s);
+  TimedChain chain(s, !f32 && variant != DMUON_VARIANT_BATCHED && tile == 512 && h.steps > 0);
     });
     if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "scale epilogue: %s", cudaGetErrorString(e));
     return DMUON_OK;
@@ -1572,12 +1625,12 @@ int dmuon_timing_get(int kind, int64_t* launches, double* ms, double* flops, dou
   int64_t n = 0;
   double t = 0, f = 0, b = 0;
   for (auto& x : g_timed) {
-    if (x.kind != kind) continue;
+    if (kind == KIND_TC_GEMM_PAIR ? !(x.kind == KIND_TC_GEMM && x.pair) : x.kind != kind) continue;
     cudaError_t e = cudaEventSynchronize(x.b);
     if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "timing event: %s", cudaGetErrorString(e));
     float d = 0.f;
     cudaEventElapsedTime(&d, x.a, x.b);
-    ++n;
+    n += x.launches;
     t += d;
     f += x.flops;
     b += x.bytes;

@@ -35,7 +35,9 @@ struct SimtGemm {
 };
 
 // Kernel classes for timing (dmuon_timing_get).
-enum KernelKind { KIND_TC_GEMM = 0, KIND_EW = 1, KIND_SIMT_GEMM = 2, KIND_OTHER = 3, KIND_COUNT = 4 };
+// KIND_TC_GEMM_PAIR is a view for dmuon_timing_get: the KIND_TC_GEMM
+// launches of the CTA-pair kernel alone.
+enum KernelKind { KIND_TC_GEMM = 0, KIND_EW = 1, KIND_SIMT_GEMM = 2, KIND_OTHER = 3, KIND_TC_GEMM_PAIR = 4 };
 
 cudaError_t launch_tc_gemm(const TcGemm& g, cudaStream_t s, int* dev_err, int num_sms);
 // Output tiles a launch of this shape processes (symmetric skipping included).
@@ -103,6 +105,9 @@ cudaError_t launch_adamw(const AdamwArgs& a, long long total_chunks, cudaStream_
 // pointer 16-byte aligned; host pointers must be mapped pinned memory).
 cudaError_t launch_copy_tables(const void* const* src, void* const* dst, long long bytes, int cnt, int num_sms,
                                cudaStream_t st);
+
+// dst[0..3] <- p0..p3 (device table written by a one-thread kernel).
+cudaError_t launch_store_ptrs(void** dst, void* p0, void* p1, void* p2, void* p3, cudaStream_t st);
 
 // One-block kernel whose only mbarrier wait can never complete; it gives up
 // after limit_ns and records kErrTimeout in *err.

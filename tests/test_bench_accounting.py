@@ -37,9 +37,10 @@ def test_profile_traffic_needs_matching_source(tmp_path, monkeypatch):
     summ = prof / "tc_gemm_pair_batch64-1024x1024.md"
     summ.write_text(f"traffic_bytes_per_launch: 1234\nkernel_source_sha256_16: {sha}\n")
     monkeypatch.setattr(bench, "ROOT", tmp_path)
-    assert bench.profile_traffic(src) == 1234.0
+    assert bench.profile_traffic(src, "batch64-1024x1024-bf16") == 1234.0
+    assert bench.profile_traffic(src, "skewed-shapes-bf16") is None  # no summary for that workload
     src.write_text("// kernel, changed\n")
-    assert bench.profile_traffic(src) is None
+    assert bench.profile_traffic(src, "batch64-1024x1024-bf16") is None
 
 
 def test_fp32_peak_from_unit_counts():
