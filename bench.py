@@ -369,6 +369,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--step-only", action="store_true",
+                    help="time the step alone: no per-kernel pass, end-to-end, AdamW or CPU baseline "
+                         "(profiler runs)")
     ap.add_argument("--cache-file", default=None,
                     help="autotune cache: loaded before the warm-up if present, saved after it "
                          "(lets a profiled run replay the plans of an unprofiled one)")
@@ -459,6 +462,18 @@ def main():
     time.sleep(0.2)
     clocks.stop()
     clk = clocks.summary(t_host0, t_host1)
+    if args.step_only:
+        ms_max = reduce_max([ms], ws, device=dev)[0]
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": round(job_value(ms_max, args.steps, ws), 4), "unit": "ms",
+                              "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+                              "ms_per_step": round(ms_max / args.steps, 4), "higher_is_better": False,
+                              "dtype": w.param_dtype, "config": {"workload": w.name, "l2": l2_note, "plans": plans},
+                              "gpu_launches_per_step": launches, "clocks": clk, "step_only": True}), flush=True)
+        if ws > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
 
     # ---------------- per-kernel timing pass: the same steps again, the
     # Newton-Schulz products of every chunk bracketed by one pair of events
@@ -539,7 +554,9 @@ def main():
         dom_kernel = ("ns_small_kernel (resident)" if variants_used == {"batched"}
                       else "tc_gemm_kernel / tc_gemm2_kernel / ns_small_kernel")
     else:
-        dom, dom_kernel, prof = simt, "simt_gemm_kernel (fp32 FFMA)", None
+        dom, prof = simt, None
+        dom_kernel = ("ns_f32_kernel (fp32 FFMA, every step in one cooperative launch)"
+                      if variants_used == {"batched"} else "simt_gemm_kernel (fp32 FFMA)")
     ach = dom["flops"] / (dom["ms"] * 1e-3) / 1e12 if dom["ms"] > 0 else 0.0
     share = round(dom["ms"] / kt_steps / ms_per_step, 3) if ms_per_step else None
     per_launch_ms = dom["ms"] / dom["launches"] if dom["launches"] else None

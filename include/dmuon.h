@@ -72,9 +72,12 @@ typedef enum dmuon_variant {
   DMUON_VARIANT_AUTO = 0,
   DMUON_VARIANT_DIRECT = 1,  /* iterate on X (m x n): 5 x (m^2 n + m^3 + m^2 n) GEMMs */
   DMUON_VARIANT_GRAM = 2,    /* iterate on Q (m x m), one m x m x n product at the end */
-  DMUON_VARIANT_BATCHED = 3  /* resident: up to 8 small matrices (m <= 128, n <= 512, bf16) per CTA,
-                                iterate, A and P in shared memory for all steps; other shapes
-                                run as AUTO */
+  DMUON_VARIANT_BATCHED = 3  /* resident, every step in one launch.  bf16, m <= 128, n <= 512: up
+                                to 8 small matrices per CTA, iterate, A and P in shared memory for
+                                all steps.  bf16, other m <= 256, n <= 1024: one CTA pair per
+                                matrix, A and P in shared memory, X streamed over k.  fp32,
+                                m <= 1024: one cooperative launch over all SMs, a grid barrier
+                                between products.  Other shapes run as AUTO */
 } dmuon_variant;
 
 /* Options of dmuon_step_ex.  Zero-initialise, then call dmuon_options_init. */
@@ -171,11 +174,23 @@ int dmuon_compute_update(const void* const* grads, void* const* momenta,
  * wide ones) is rejected with DMUON_ERR_INVALID before any launch.  The
  * first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
- * capture.  It uses the plan the autotuner cached for this shape (count 1)
- * when there is one, else the direct form; it never autotunes.  All calls
- * share the one array and it keeps the last call's contents (each call
- * clears the words it reads before writing them): calls whose GPU work
- * overlaps, e.g. on two streams without ordering between them, race.
+ * capture.  The address is kept for the life of the process, so
+ * cudaDeviceReset while the library is loaded is not supported.
+ * Plan: opts->variant == DMUON_VARIANT_BATCHED runs the resident kernel when
+ * the shape fits it (bf16, m <= 128, n <= 512); otherwise the call uses the
+ * plan the autotuner cached for this shape (count 1) when there is one, else
+ * the direct form; it never autotunes.
+ * All calls share the one array and it keeps the last call's contents (each
+ * call writes every word it reads before reading it, except the error word
+ * below): calls whose GPU work overlaps, e.g. on two streams without
+ * ordering between them, race.
+ * A bounded device-side wait that gives up (DMUON_ERR_DEVICE_TIMEOUT) leaves
+ * its code in an error word of the array; the call that launched it has
+ * already returned.  Each call first reads that word (4 bytes, on the
+ * per-thread default stream, so it does not wait for `stream`), except while
+ * `stream` is being captured; if it holds a code, the call clears it and
+ * returns DMUON_ERR_DEVICE_TIMEOUT without launching anything.  A timeout is
+ * therefore reported by a later call of this entry point.
  * Calls no cudaMalloc, cudaFree or other allocating routine.
  */
 int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows, int64_t cols, float mu,
@@ -227,12 +242,17 @@ int dmuon_set_workspace(void* dev_ptr, size_t bytes);
 int dmuon_workspace_size(const int64_t* shapes, int count, int param_dtype, size_t* bytes);
 
 /*
- * Kernel timing for benchmarks.  While enabled, the library brackets every
- * launch with CUDA events on the stream it launches on.  dmuon_timing_get
- * synchronises those events and returns, for kernel class `kind`
- * (0 = tensor-core GEMM, 1 = momentum/normalise, 2 = SIMT GEMM, 3 = other),
- * the number of launches, their summed device time in ms, the algorithmic
- * FLOPs (GEMM: 2*M*N*K*batch) and algorithmic bytes (elementwise kernels).
+ * Kernel timing for benchmarks.  While enabled, the library records CUDA
+ * events on the stream it launches on: the Newton-Schulz products of one
+ * chunk of a shape group are bracketed as one chain (one pair of events
+ * around all of them, none between two of its kernels, so short launches are
+ * not stretched by the timing itself); every other launch gets its own pair.
+ * dmuon_timing_get synchronises those events and returns, for kernel class
+ * `kind` (0 = tensor-core GEMM, 1 = momentum, 2 = SIMT GEMM, 3 = other,
+ * 4 = the tensor-core GEMM chains of the CTA-pair kernel alone, a subset of
+ * 0), the number of launches, their summed device time in ms, the
+ * algorithmic FLOPs (GEMM: 2*M*N*K*batch over the computed tiles) and
+ * algorithmic bytes (elementwise kernels).
  */
 void dmuon_timing_enable(int enable);
 void dmuon_timing_reset(void);

@@ -237,6 +237,13 @@ bool fault_alloc() {
   return f && strstr(f, "alloc");
 }
 
+// DMUON_FAULT=wait: dmuon_compute_update_noalloc ends with a bounded wait
+// that nothing completes (20 ms), so its error word records a timeout.
+bool fault_wait() {
+  const char* f = getenv("DMUON_FAULT");
+  return f && strstr(f, "wait");
+}
+
 int ensure_ws(DeviceCtx& c, size_t bytes, cudaStream_t s) {
   if (g_ext_ptr) {
     if (bytes > g_ext_bytes)
@@ -317,7 +324,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Scratch layout of one chunk of `cnt` matrices.
 struct Layout {
-  size_t X0, Xp, Xq, A, Bm, P, Q0, Q1, T, partials, s, s2, total;
+  size_t X0, Xp, Xq, A, Bm, P, Q0, Q1, T, partials, s, s2, sync, total;
 };
 
 Layout make_layout(const Geo& g, int cnt, int nblk) {
@@ -342,6 +349,7 @@ Layout make_layout(const Geo& g, int cnt, int nblk) {
   L.partials = take(static_cast<size_t>(cnt) * nblk * sizeof(float));
   L.s = take(static_cast<size_t>(cnt) * sizeof(float));
   L.s2 = take(static_cast<size_t>(cnt) * sizeof(float));
+  L.sync = take(16);  // grid-barrier words of the fp32 resident kernel
   L.total = off;
   return L;
 }
@@ -466,6 +474,7 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
   void* X0 = at<void>(ch, ch.L.X0);
   Epilogue fin = fin_in;
   int rc;
+  TimedChain chain(s, !f32 && variant != DMUON_VARIANT_BATCHED && tile == 512 && h.steps > 0);
   if (h.steps == 0) {  // O = X0 = s U; the kernel folds s in
     fin.alpha = 1.f;
     fin.alpha_vec = nullptr;
@@ -473,12 +482,31 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
     fin.C = nullptr;
     cudaError_t e = launch_k(KIND_OTHER, 0.0, 0.0, s, [&] {
       return launch_scale_epilogue(X0, g.ldx, f32, m, n, cnt, sv, fin, s);
-  TimedChain chain(s, !f32 && variant != DMUON_VARIANT_BATCHED && tile == 512 && h.steps > 0);
     });
     if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "scale epilogue: %s", cudaGetErrorString(e));
     return DMUON_OK;
   }
-  if (variant == DMUON_VARIANT_BATCHED) {  // resident small-matrix kernel (bf16 only)
+  if (variant == DMUON_VARIANT_BATCHED && f32) {  // fp32: every step in one cooperative launch
+    NsF32 a{static_cast<const float*>(X0), at<float>(ch, ch.L.Xp), at<float>(ch, ch.L.Xq), at<float>(ch, ch.L.A),
+            at<float>(ch, ch.L.Bm), g.ldx, g.ldm, sx, sq, sv, s2v, cnt, m, n, h.steps, h.a, h.b, h.c, fin,
+            at<unsigned>(ch, ch.L.sync)};
+    const double T = (m + 15) / 16;
+    const double symf = (T * (T + 1) / 2) / (T * T);
+    const double fl = 2.0 * h.steps * cnt * (symf * m * static_cast<double>(m) * n + symf * m * static_cast<double>(m) * m +
+                                            m * static_cast<double>(m) * n);
+    cudaError_t e = launch_k(KIND_SIMT_GEMM, fl, 0.0, s, [&] { return launch_ns_f32(a, s, c.err_dev, c.num_sms); });
+    if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "fp32 resident kernel: %s", cudaGetErrorString(e));
+    return DMUON_OK;
+  }
+  if (variant == DMUON_VARIANT_BATCHED && !ns_small_supported(m, n)) {  // bf16, medium: one CTA pair per matrix
+    cudaError_t e = launch_k(KIND_TC_GEMM, ns_mid_flops(m, n, h.steps, cnt), 0.0, s, [&] {
+      return launch_ns_mid(X0, at<void>(ch, ch.L.Xp), g.ldx, sv, s2v, cnt, m, n, h.steps, h.a, h.b, h.c, fin, s,
+                           c.err_dev, c.num_sms);
+    });
+    if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "resident medium-matrix kernel: %s", cudaGetErrorString(e));
+    return DMUON_OK;
+  }
+  if (variant == DMUON_VARIANT_BATCHED) {  // resident small-matrix kernel (bf16)
     cudaError_t e = launch_k(KIND_TC_GEMM, 2.0 * h.steps * (2.0 * 128 * 128 * g.n + 2.0 * 128 * 128 * 128) *
                                                ((cnt + ns_small_group(m) - 1) / ns_small_group(m)),
                              0.0, s, [&] {
@@ -637,6 +665,14 @@ int forced_tile() {
   return 0;
 }
 
+// The resident variant (DMUON_VARIANT_BATCHED) for this dtype and shape:
+// bf16 stacks small matrices in shared memory and TMEM (m <= 128, n <= 512)
+// or gives a medium matrix a CTA pair (m <= 256, n <= 1024); fp32 runs every
+// step in one cooperative launch (m <= 1024).
+bool resident_supported(bool f32, int m, int n) {
+  return f32 ? ns_f32_supported(m, n) : (ns_small_supported(m, n) || ns_mid_supported(m, n));
+}
+
 double gate_tol() {
   const char* g = getenv("DMUON_GATE");
   return g ? atof(g) : 2e-2;
@@ -720,7 +756,7 @@ int autotune(DeviceCtx& c, const Chunk& ch, bool f32, const Hyper& h, int forced
   }
   for (int v : vars)
     for (int t : tiles) cands.push_back({v, t});
-  if (!f32 && ns_small_supported(g.m, g.n) &&
+  if (resident_supported(f32, g.m, g.n) && h.steps > 0 &&
       (forced_variant == DMUON_VARIANT_AUTO || forced_variant == DMUON_VARIANT_BATCHED))
     cands.push_back({DMUON_VARIANT_BATCHED, 128});
   if (forced_variant == DMUON_VARIANT_BATCHED && !cands.empty() && cands.back().first == DMUON_VARIANT_BATCHED)
@@ -884,9 +920,9 @@ int run_step(Request& r) {
     {
       std::lock_guard<std::mutex> lk2(g_cache_mu);
       auto it = g_cache.find(key);
-      // a forced variant the shape cannot take (the resident kernel needs
-      // bf16, m <= 128, n <= 512) runs as planned for AUTO
-      const bool forced_ok = r.o.variant != DMUON_VARIANT_BATCHED || (!f32 && ns_small_supported(geos[k].m, geos[k].n));
+      // a forced variant the shape cannot take (see resident_supported)
+      // runs as planned for AUTO
+      const bool forced_ok = r.o.variant != DMUON_VARIANT_BATCHED || resident_supported(f32, geos[k].m, geos[k].n);
       const int want = forced_ok ? r.o.variant : DMUON_VARIANT_AUTO;
       if (it != g_cache.end() && (want == DMUON_VARIANT_AUTO || it->second.variant == want)) {
         gr.plan = it->second;
@@ -1277,13 +1313,20 @@ int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows,
   int rc = validate(r);
   if (rc) return rc;
   const bool f32 = o.param_dtype == DMUON_F32;
-  // plan: the one the autotuner cached for this shape, else the direct form
+  const Geo g = make_geo(rows, cols, f32);
+  // plan: the resident kernel when it is asked for and the shape fits it;
+  // else the plan the autotuner cached for this shape (count 1), else the
+  // direct form (a forced variant the shape cannot take runs as AUTO)
   Plan plan;
-  if (o.variant == DMUON_VARIANT_DIRECT || o.variant == DMUON_VARIANT_GRAM) plan.variant = o.variant;
-  {
+  if (o.variant == DMUON_VARIANT_BATCHED && resident_supported(f32, g.m, g.n)) {
+    plan.variant = DMUON_VARIANT_BATCHED;
+    plan.tile = 128;
+  } else {
+    const int want = o.variant == DMUON_VARIANT_BATCHED ? DMUON_VARIANT_AUTO : o.variant;
+    if (want == DMUON_VARIANT_DIRECT || want == DMUON_VARIANT_GRAM) plan.variant = want;
     std::lock_guard<std::mutex> lk(g_cache_mu);
     auto it = g_cache.find(Key{rows, cols, f32 ? 1 : 0, ns_steps, 1});
-    if (it != g_cache.end() && (o.variant == DMUON_VARIANT_AUTO || it->second.variant == o.variant)) plan = it->second;
+    if (it != g_cache.end() && (want == DMUON_VARIANT_AUTO || it->second.variant == want)) plan = it->second;
   }
   void* base = nullptr;
   int dev = 0;
@@ -1291,7 +1334,6 @@ int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows,
   if (rc) return rc;
   int sms = 0;
   CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  const Geo g = make_geo(rows, cols, f32);
   const int nblk = momentum_partials(g.rows, g.cols);
   const Layout L = make_layout(g, 1, nblk);
   const size_t header = 256;  // 4 pointer slots and the device error word
@@ -1302,10 +1344,27 @@ int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows,
                 (long long)rows, (long long)cols, f32 ? "fp32" : "bf16", need, kStaticScratchBytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* sb = static_cast<uint8_t*>(base);
-  void* tables[4] = {gp, momentum, nullptr, out};
-  CUDA_TRY(cudaMemcpyAsync(sb, tables, sizeof(tables), cudaMemcpyHostToDevice, s));
   int* dev_err = reinterpret_cast<int*>(sb + 64);
-  CUDA_TRY(cudaMemsetAsync(dev_err, 0, sizeof(int), s));  // the only word read before it is written
+  // A bounded device wait that gave up in an earlier call left its code in
+  // the error word, which no call clears unread.  The word is read here
+  // (4 bytes on the per-thread stream, which does not wait for `stream`),
+  // except while `stream` is being captured; a code found is reported now,
+  // and the word cleared, before any launch.
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  CUDA_TRY(cudaStreamIsCapturing(s, &cap));
+  if (cap == cudaStreamCaptureStatusNone) {
+    int word = 0;
+    CUDA_TRY(cudaMemcpyAsync(&word, dev_err, sizeof(int), cudaMemcpyDeviceToHost, cudaStreamPerThread));
+    CUDA_TRY(cudaStreamSynchronize(cudaStreamPerThread));
+    if (word != 0) {
+      CUDA_TRY(cudaMemsetAsync(dev_err, 0, sizeof(int), s));
+      return fail(DMUON_ERR_DEVICE_TIMEOUT, "a device-side wait of an earlier dmuon_compute_update_noalloc call timed out");
+    }
+  }
+  // pointer table (G, B, W, O) written on the device from kernel arguments
+  void** dtab = reinterpret_cast<void**>(sb);
+  cudaError_t e = launch_k(KIND_OTHER, 0.0, 0.0, s, [&] { return launch_store_ptrs(dtab, gp, momentum, nullptr, out, s); });
+  if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "pointer table: %s", cudaGetErrorString(e));
   DeviceCtx c;  // launch parameters only: nothing is allocated for it
   c.device = dev;
   c.num_sms = sms;
@@ -1315,7 +1374,6 @@ int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows,
   ch.cnt = 1;
   ch.base = sb + header;
   ch.L = L;
-  void** dtab = reinterpret_cast<void**>(sb);
   ch.Gt = dtab;
   ch.Bt = dtab + 1;
   ch.Wt = dtab + 2;
@@ -1330,7 +1388,13 @@ int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows,
   fin.transposed = g.transposed;
   fin.ldw = g.cols;
   fin.w_f32 = f32;
-  return run_ns(c, ch, f32, plan.variant, plan.tile, r.h, fin, 1, s);
+  rc = run_ns(c, ch, f32, plan.variant, plan.tile, r.h, fin, 1, s);
+  if (rc) return rc;
+  if (fault_wait()) {  // DMUON_FAULT=wait: a bounded wait that runs out, as a stalled pipeline would
+    e = launch_wait_selftest(dev_err, 20000000ull, s);
+    if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "injected wait: %s", cudaGetErrorString(e));
+  }
+  return DMUON_OK;
 }
 
 int dmuon_gemm_bf16(const void* A, int64_t lda, int64_t sa, const void* B, int64_t ldb, int64_t sb, int b_kmajor,

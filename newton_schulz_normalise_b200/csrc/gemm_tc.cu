@@ -714,6 +714,12 @@ cudaError_t launch_pair(const TcGemm& g, cudaStream_t s, int* dev_err, int num_s
 
 }  // namespace
 
+bool tensor_map_bf16(CUtensorMap* m, const void* base, long long inner, long long outer, int batch, long long ld,
+                     long long bstride, int box_inner, int box_outer) {
+  if (get_encode() != cudaSuccess) return false;
+  return make_map(m, base, inner, outer, batch, ld, bstride, box_inner, box_outer);
+}
+
 long long tc_gemm_tiles(int M, int N, int batch, int tile, bool sym) {
   if (tile == 512) return tiles_per_matrix(M, N, P_BM, P_BN, sym) * batch;
   return tiles_per_matrix(M, N, BM, tile == 128 ? 128 : 256, sym) * batch;

@@ -40,6 +40,11 @@ struct SimtGemm {
 enum KernelKind { KIND_TC_GEMM = 0, KIND_EW = 1, KIND_SIMT_GEMM = 2, KIND_OTHER = 3, KIND_TC_GEMM_PAIR = 4 };
 
 cudaError_t launch_tc_gemm(const TcGemm& g, cudaStream_t s, int* dev_err, int num_sms);
+// 3-D bf16 tensor map {inner, outer, batch} with a 128-byte swizzle and
+// zero fill outside the extents (row stride ld, batch stride bstride, in
+// elements; box box_inner x box_outer x 1).
+bool tensor_map_bf16(CUtensorMap* m, const void* base, long long inner, long long outer, int batch, long long ld,
+                     long long bstride, int box_inner, int box_outer);
 // Output tiles a launch of this shape processes (symmetric skipping included).
 long long tc_gemm_tiles(int M, int N, int batch, int tile, bool sym);
 cudaError_t launch_simt_gemm(const SimtGemm& g, cudaStream_t s);
@@ -79,6 +84,38 @@ bool ns_small_supported(int m, int n);
 int ns_small_group(int m);
 cudaError_t launch_ns_small(const void* X0, long long ldx, const float* s, const float* s2, int cnt, int m, int n,
                             int steps, float a, float b, float c, const Epilogue& fin, cudaStream_t st, int* err);
+
+// fp32 Newton-Schulz, direct form, every step of `cnt` same-shape matrices in
+// one cooperative launch (one CTA per SM, grid barrier between products);
+// ends with `fin`.  X0/Xp/Xq: [cnt][m][ldx], A/P: [cnt][m][ldm] scratch; sync:
+// three words of scratch.
+struct NsF32 {
+  const float* X0;
+  float* Xp;
+  float* Xq;
+  float* A;
+  float* P;
+  long long ldx, ldm, sx, sq;  // row strides and per-matrix strides (elements)
+  const float* s;
+  const float* s2;
+  int cnt, m, n, steps;
+  float a, b, c;
+  Epilogue fin;
+  unsigned* sync;
+};
+bool ns_f32_supported(int m, int n);
+cudaError_t launch_ns_f32(const NsF32& g, cudaStream_t st, int* err, int num_sms);
+
+// Resident Newton-Schulz for medium bf16 matrices (128 < m <= 256, or m <= 128
+// with 512 < n; n <= 1024), direct form: one CTA pair per matrix, A and P in
+// shared memory for all steps, X streamed over k from the scratch.  X0 is
+// read, never written; Xw ([cnt][m][ldx], same layout) holds the iterate
+// from the second step on.  Ends with `fin`.
+bool ns_mid_supported(int m, int n);
+cudaError_t launch_ns_mid(const void* X0, void* Xw, long long ldx, const float* s, const float* s2, int cnt, int m,
+                          int n, int steps, float a, float b, float c, const Epilogue& fin, cudaStream_t st, int* err,
+                          int num_sms);
+double ns_mid_flops(int m, int n, int steps, int cnt);
 
 // AdamW over `count` tensors in one launch (see kernels_ew.cu).  Tables are
 // device arrays; chunk_start[t] is the first chunk of tensor t (prefix sums of

@@ -268,6 +268,16 @@ __global__ void wait_selftest_kernel(int* err, unsigned long long limit_ns) {
     *reinterpret_cast<volatile int*>(err) = kErrTimeout;
 }
 
+// Writes four pointers, passed by value, into a device table: a pointer
+// table built on the device from kernel arguments, with no host buffer that
+// must outlive the call.
+__global__ void store_ptrs_kernel(void** dst, void* p0, void* p1, void* p2, void* p3) {
+  dst[0] = p0;
+  dst[1] = p1;
+  dst[2] = p2;
+  dst[3] = p3;
+}
+
 // Copies cnt buffers of `bytes` each, dst[l] <- src[l], through the SMs.
 // Either side may be pinned host memory mapped into the device's address
 // space: the host I/O pipeline gathers gradients from, and scatters
@@ -420,6 +430,11 @@ cudaError_t launch_copy_tables(const void* const* src, void* const* dst, long lo
   dim3 grid(static_cast<unsigned>(bx), cnt);
   copy_tables_kernel<<<grid, COPY_THREADS, 0, st>>>(reinterpret_cast<const uint4* const*>(src),
                                                     reinterpret_cast<uint4* const*>(dst), nvec);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_store_ptrs(void** dst, void* p0, void* p1, void* p2, void* p3, cudaStream_t st) {
+  store_ptrs_kernel<<<1, 1, 0, st>>>(dst, p0, p1, p2, p3);
   return cudaGetLastError();
 }
 

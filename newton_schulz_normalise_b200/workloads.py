@@ -81,6 +81,10 @@ WORKLOADS = {
     # Llama-style 8B matrix set: 32 layers of q, k, v, o, gate, up, down
     "llama8b-matrices-bf16": Workload(
         "llama8b-matrices-bf16", _LLAMA8B_LAYER, seed=4, interleave=32),
+    # one layer of that set (every shape and product of it at 1/32 of the
+    # size: small enough for profiler captures, 1.75 GB > L2)
+    "llama8b-layer-bf16": Workload(
+        "llama8b-layer-bf16", _LLAMA8B_LAYER, seed=4, interleave=1),
 }
 
 _DT = {"bf16": torch.bfloat16, "f32": torch.float32}

@@ -223,3 +223,93 @@ def test_forced_tile_matches_oracle(dmuon_lib, monkeypatch, tile):
         e = rel_fro(to64(Os[i]), Oo)
         assert e <= BF16_TOL, (shapes[i], tile, e)
         check_momentum(Bn[i], Gs[i], Ms[i], 0.95)
+
+
+@pytest.mark.parametrize("shapes", [[(256, 512)], [(300, 100)] * 2, [(1, 64)] * 3, [(17, 33)] * 4, [(130, 70)],
+                                    [(64, 2100)], [(1000, 1024)]],
+                         ids=["256x512", "300x100x2", "1x64x3", "17x33x4", "130x70", "64x2100", "1000x1024"])
+def test_fp32_resident_kernel(dmuon_lib, shapes):
+    """fp32: every Newton-Schulz step in one cooperative launch (grid barrier
+    between products) against the oracle at the fp32 bar and against the
+    separate-launch SIMT form it restates; then its fused parameter write.
+    64 x 2100 stages X X^T's k in more than one chunk; 1000 x 1024 fills the
+    largest m the kernel takes."""
+    Ws, Gs, Ms = make_inputs(shapes, seed=93, pdt="f32", m_std=0.02, g_std=0.02)
+    Ob, Bb = gpu_update(dmuon_lib, Gs, Ms, variant="batched")
+    Od, _ = gpu_update(dmuon_lib, Gs, Ms, variant="direct")
+    for i in range(len(shapes)):
+        _, Oo = oracle_update(Gs[i], Ms[i])
+        assert rel_fro(to64(Ob[i]), Oo) <= F32_TOL, (i, rel_fro(to64(Ob[i]), Oo))
+        assert rel_fro(to64(Ob[i]), to64(Od[i])) <= 1e-5, i
+        check_momentum(Bb[i], Gs[i], Ms[i], 0.95)
+    Wg, _ = gpu_step(dmuon_lib, Ws, Gs, Ms, variant="batched")
+    for i, (r, c) in enumerate(shapes):
+        w_apply = ora.apply_update(to64(Ws[i]), to64(Ob[i]), 0.02, 0.1)
+        terms = np.abs(0.998 * to64(Ws[i])) + np.abs(0.02 * ora.rms_scale(r, c) * to64(Ob[i]))
+        assert np.all(np.abs(to64(Wg[i]) - w_apply) <= terms * 2.0 ** -21), i
+
+
+@pytest.mark.parametrize("steps", [1, 2, 7])
+def test_fp32_resident_steps(dmuon_lib, steps):
+    shapes = [(96, 200), (200, 96)]
+    Ws, Gs, Ms = make_inputs(shapes, seed=94, pdt="f32", m_std=0.02, g_std=0.02)
+    Os, _ = gpu_update(dmuon_lib, Gs, Ms, steps=steps, variant="batched")
+    for i in range(len(shapes)):
+        _, Oo = oracle_update(Gs[i], Ms[i], steps=steps)
+        assert rel_fro(to64(Os[i]), Oo) <= F32_TOL, (steps, i)
+
+
+def test_fp32_resident_nonfinite_stays_in_its_matrix(dmuon_lib):
+    shapes = [(128, 256)] * 3
+    Ws, Gs, Ms = make_inputs(shapes, seed=95, pdt="f32", m_std=0.02, g_std=0.02)
+    Gs[1] = Gs[1].clone()
+    Gs[1][3, 4] = float("nan")
+    Os, _ = gpu_update(dmuon_lib, Gs, Ms, variant="batched")
+    assert not torch.isfinite(Os[1]).any()
+    for i in (0, 2):
+        _, Oo = oracle_update(Gs[i], Ms[i])
+        assert rel_fro(to64(Os[i]), Oo) <= F32_TOL, i
+
+
+@pytest.mark.parametrize("shapes", [[(256, 1024)] * 3, [(200, 700)] * 2, [(1024, 256)], [(129, 300)], [(100, 900)],
+                                    [(256, 256)] * 2, [(250, 1000)]],
+                         ids=["256x1024x3", "200x700x2", "1024x256", "129x300", "100x900", "256x256x2", "250x1000"])
+def test_resident_medium_kernel(dmuon_lib, shapes):
+    """The medium resident kernel (one CTA pair per matrix, A and P on chip,
+    X streamed over k, all steps in one launch) against the oracle and the
+    direct form it restates; then its fused parameter write."""
+    Ws, Gs, Ms = make_inputs(shapes, seed=97, m_std=1e-3)
+    Ob, Bb = gpu_update(dmuon_lib, Gs, Ms, variant="batched")
+    Od, _ = gpu_update(dmuon_lib, Gs, Ms, variant="direct")
+    for i in range(len(shapes)):
+        _, Oo = oracle_update(Gs[i], Ms[i])
+        assert rel_fro(to64(Ob[i]), Oo) <= BF16_TOL, (i, rel_fro(to64(Ob[i]), Oo))
+        assert rel_fro(to64(Ob[i]), to64(Od[i])) <= 1e-2, i
+        check_momentum(Bb[i], Gs[i], Ms[i], 0.95)
+    Wg, _ = gpu_step(dmuon_lib, Ws, Gs, Ms, variant="batched")
+    for i, (r, c) in enumerate(shapes):
+        w_apply = ora.apply_update(to64(Ws[i]), to64(Ob[i]), 0.02, 0.1)
+        terms = np.abs(0.998 * to64(Ws[i])) + np.abs(0.02 * ora.rms_scale(r, c) * to64(Ob[i]))
+        assert np.all(np.abs(to64(Wg[i]) - w_apply) <= np.abs(w_apply) * 2.0 ** -8 + terms * 1e-6), i
+
+
+@pytest.mark.parametrize("steps", [1, 2, 7])
+def test_resident_medium_steps(dmuon_lib, steps):
+    shapes = [(256, 1024), (700, 180)]
+    Ws, Gs, Ms = make_inputs(shapes, seed=98, m_std=1e-3)
+    Os, _ = gpu_update(dmuon_lib, Gs, Ms, steps=steps, variant="batched")
+    for i in range(len(shapes)):
+        _, Oo = oracle_update(Gs[i], Ms[i], steps=steps)
+        assert rel_fro(to64(Os[i]), Oo) <= BF16_TOL, (steps, i)
+
+
+def test_resident_medium_nonfinite_stays_in_its_matrix(dmuon_lib):
+    shapes = [(256, 1024)] * 3
+    Ws, Gs, Ms = make_inputs(shapes, seed=99)
+    Gs[1] = Gs[1].clone()
+    Gs[1][9, 9] = float("nan")
+    Os, _ = gpu_update(dmuon_lib, Gs, Ms, variant="batched")
+    assert not torch.isfinite(Os[1]).any()
+    for i in (0, 2):
+        _, Oo = oracle_update(Gs[i], Ms[i])
+        assert rel_fro(to64(Os[i]), Oo) <= BF16_TOL, i

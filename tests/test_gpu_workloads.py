@@ -1,18 +1,21 @@
 """Full-size parity on every workload, in the launch configuration bench.py
-times: one dmuon_step call over the whole parameter set.
+times: one call over the whole parameter set.
 
-* The update O is checked on sampled matrices (first and last of every shape
-  group) against the fp64 oracle.  A weight write W' = (1-lr*wd) W - lr*s*O
-  cannot resolve O when W dominates, so the step runs on a copy of the
-  workload with W = 0: then W' = -lr*s*O up to one bf16 rounding (2^-9).
-* The momentum buffer is checked on every element of every matrix against
-  an independent fp64 torch expression on the harness side.
+* dmuon_compute_update runs on the whole set and returns the fp32 update O of
+  every matrix.  O is checked on sampled matrices (first and last of every
+  shape group) against the fp64 oracle at the stated bar: relative Frobenius
+  error <= 3e-2 on the bf16 path, <= 1e-4 on the fp32 path.
+* The momentum buffer is checked on every element of every matrix against an
+  independent fp64 torch expression on the harness side.
+* dmuon_step_ex then runs on the same inputs (the bench's call, with the
+  plans the first call cached).  Its fused parameter write is checked on
+  every element of every matrix against W' = (1 - lr wd) W - lr s O computed
+  in fp64 from the O above: within one rounding to the parameter dtype plus
+  the fp32 evaluation of the two-term sum.
 For wide samples the oracle uses its Gram-space form, which its pins hold to
 within 1e-10 of the direct form; the direct form is too slow in fp64 at
 4096 x 14336.
 """
-import dataclasses
-
 import numpy as np
 import pytest
 import torch
@@ -34,30 +37,52 @@ def _samples(shapes):
     return sorted(set(first.values()) | set(last.values()))
 
 
+def _check_momentum(Bn, G, M0, mu, i):
+    ref = mu * M0.double() + G.double()
+    bound = 1e-6 * ((mu * M0.double()).abs() + G.double().abs()) + 1e-30
+    assert bool(((Bn.double() - ref).abs() <= bound).all()), f"momentum matrix {i}"
+
+
 @pytest.mark.parametrize("name", NAMES)
 def test_workload_full_size(dmuon_lib, name):
-    w = dataclasses.replace(wl.WORKLOADS[name], w_std=0.0)  # W = 0 copy, same launch config
+    w = wl.WORKLOADS[name]
     f32 = w.param_dtype == "f32"
     tol = 1e-4 if f32 else 3e-2
     Ws, Gs, Ms = wl.generate(w, device="cuda")
     shapes = w.shapes()
     samples = _samples(shapes)
     host = {i: (Gs[i].double().cpu().numpy(), Ms[i].double().cpu().numpy()) for i in samples}
-    # momentum reference for every matrix, fp64 on the device (harness side)
-    mom_ref = [w.mu * m.double() + g.double() for g, m in zip(Gs, Ms)]
-    mom_bound = [1e-6 * ((w.mu * m.double()).abs() + g.double().abs()) for g, m in zip(Gs, Ms)]
-    dmuon_lib.dmuon_step_ex(Ws, Gs, Ms, w.lr, w.wd, w.mu, w.ns_steps)
+    W0 = [x.clone() for x in Ws]
+    M0 = [x.clone() for x in Ms]
+    Os = [torch.empty(x.shape, device="cuda", dtype=torch.float32) for x in Ws]
+
+    # ---- the update O of every matrix (first call: plans tuned and cached)
+    dmuon_lib.dmuon_compute_update(Gs, Ms, Os, w.mu, w.ns_steps)
     torch.cuda.synchronize()
     for i in range(len(shapes)):
-        err = (Ms[i].double() - mom_ref[i]).abs()
-        assert bool((err <= mom_bound[i] + 1e-30).all()), f"momentum matrix {i}"
-    del mom_ref, mom_bound
+        _check_momentum(Ms[i], Gs[i], M0[i], w.mu, i)
     for i in samples:
         r, c = shapes[i]
         G, M = host[i]
         variant = "gram" if max(r, c) >= 2 * min(r, c) else "direct"
         _, O_ora = ora.muon_update(G, M, w.mu, w.ns_steps, 1e-7, True, variant)
-        O_gpu = -Ws[i].double().cpu().numpy() / (w.lr * ora.rms_scale(r, c))
+        O_gpu = Os[i].double().cpu().numpy()
         e = np.linalg.norm(O_gpu - O_ora) / np.linalg.norm(O_ora)
-        # bf16 storage of W' adds at most 2^-9 relative
-        assert e <= tol + (0 if f32 else 2.0 ** -9), (name, i, (r, c), e)
+        assert e <= tol, (name, i, (r, c), e)
+
+    # ---- the bench's call on the same inputs: fused scale, decay and write
+    for m, m0 in zip(Ms, M0):
+        m.copy_(m0)
+    dmuon_lib.dmuon_step_ex(Ws, Gs, Ms, w.lr, w.wd, w.mu, w.ns_steps)
+    torch.cuda.synchronize()
+    decay = 1.0 - np.float32(w.lr) * np.float32(w.wd)  # as the library forms it, in fp32
+    unit = 2.0 ** -24 if f32 else 2.0 ** -8  # one rounding to the parameter dtype, relative
+    for i, (r, c) in enumerate(shapes):
+        _check_momentum(Ms[i], Gs[i], M0[i], w.mu, i)
+        lr_s = float(np.float32(w.lr) * np.float32(0.2) * np.sqrt(np.float32(max(r, c))))
+        dw = float(decay) * W0[i].double()
+        do = lr_s * Os[i].double()
+        ref = dw - do
+        bound = unit * ref.abs() + 2.0 ** -22 * (dw.abs() + do.abs()) + 1e-30
+        err = (Ws[i].double() - ref).abs()
+        assert bool((err <= bound).all()), (name, i, (r, c), float((err / bound).max()))
