@@ -46,30 +46,52 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;  // 64 bf16 = 128 bytes = one swizzle row
 
-// Tile t of a launch -> (matrix l, tile row tm, tile column tn).  With sym
-// the result is symmetric and only blocks on or above the block diagonal run:
-// row tm holds the tiles tn >= floor(tm*bm/bn).  Tiles strictly above it
-// (tn > floor(tm*bm/bn)) are also stored mirrored; diagonal blocks are
-// computed in full and stored as they are, so every element is written once.
+// Tile t of a launch -> (matrix l, tile row tm, tile column tn).
+// Tiles are taken in bands of RB tile rows, column by column inside a band,
+// so the ~74-148 tiles in flight at once cover a few rows and a few columns
+// (their operand rows and columns stay in L2) instead of one or two whole
+// tile rows, which re-read the right operand from DRAM once per tile row
+// when it is wide.  With sym the result is symmetric and only blocks on or
+// above the block diagonal run: row tm holds the tiles tn >= first(tm) =
+// floor(tm*bm/bn), i.e. column tn holds the rows tm < ceil((tn+1)*bn/bm).
+// Tiles strictly above it (tn > first(tm)) are also stored mirrored;
+// diagonal blocks are computed in full and stored as they are, so every
+// element is written once.  The order changes nothing in any tile's result.
+constexpr int RB = 8;  // tile rows per band
+
+__host__ __device__ __forceinline__ int sym_rows_below(int tn, int bm, int bn) {  // rows tm with first(tm) <= tn
+  return ((tn + 1) * bn + bm - 1) / bm;
+}
+
 __device__ __forceinline__ void decode_tile(long long t, long long per_mat, int tiles_m, int tiles_n, int bm,
                                             int bn, bool sym, int& l, int& tm, int& tn, bool& mirror) {
   l = static_cast<int>(t / per_mat);
   long long u = t % per_mat;
   mirror = false;
-  if (!sym) {
-    tm = static_cast<int>(u / tiles_n);
-    tn = static_cast<int>(u % tiles_n);
-    return;
-  }
-  for (tm = 0; tm < tiles_m; ++tm) {
-    const int first = (tm * bm) / bn;
-    const int cnt = tiles_n - first;
-    if (u < cnt) {
-      tn = first + static_cast<int>(u);
-      mirror = tn > first;
-      return;
+  for (int r0 = 0; r0 < tiles_m; r0 += RB) {
+    const int r1 = r0 + RB < tiles_m ? r0 + RB : tiles_m;
+    if (!sym) {
+      const long long band = static_cast<long long>(r1 - r0) * tiles_n;
+      if (u < band) {
+        tn = static_cast<int>(u / (r1 - r0));
+        tm = r0 + static_cast<int>(u % (r1 - r0));
+        return;
+      }
+      u -= band;
+      continue;
     }
-    u -= cnt;
+    for (int c = (r0 * bm) / bn; c < tiles_n; ++c) {
+      int hi = sym_rows_below(c, bm, bn);
+      hi = hi < r1 ? hi : r1;
+      const int cnt = hi - r0;
+      if (u < cnt) {
+        tn = c;
+        tm = r0 + static_cast<int>(u);
+        mirror = tn > (tm * bm) / bn;
+        return;
+      }
+      u -= cnt;
+    }
   }
   tm = tiles_m - 1;  // not reached for t < per_mat * batch
   tn = tiles_n - 1;
@@ -182,6 +204,82 @@ __device__ __forceinline__ void store_tile_staged(const Epilogue& e, const CUten
       bulk_commit();
     }
     ++st.it;
+  }
+}
+
+// ---------------------------------------------------------------- transposed parameter write
+// EPI_APPLY of a bf16 parameter stored as the transpose of the iterate (a
+// tall weight): iterate element (row, col) updates W[col][row].  Per 32 x 32
+// chunk the warp moves the W box (32 rows of W, 64 bytes each) through a
+// 2 KB staging buffer with 16-byte coalesced loads and stores: 8 memory
+// instructions per lane and chunk instead of one 2-byte load and store per
+// element.  In the buffer, lane r (iterate row) updates column r of every box
+// row: two lanes per 4-byte word, no bank conflict.
+__device__ __forceinline__ void box_rw(uint8_t* box, __nv_bfloat16* W, long long ldw, int wr0, int wc0, int nrows,
+                                       int ncols, bool vec, bool load, int lane) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int idx = q * 32 + lane;
+    const int br = idx >> 2, seg = idx & 3;
+    uint4* sp = reinterpret_cast<uint4*>(box + br * 64 + seg * 16);
+    if (br >= nrows) continue;
+    __nv_bfloat16* gp = W + static_cast<long long>(wr0 + br) * ldw + wc0 + seg * 8;
+    if (vec && seg * 8 + 8 <= ncols) {
+      if (load)
+        *sp = *reinterpret_cast<const uint4*>(gp);
+      else
+        *reinterpret_cast<uint4*>(gp) = *sp;
+    } else {
+      __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(sp);
+      for (int t = 0; t < 8; ++t)
+        if (seg * 8 + t < ncols) {
+          if (load)
+            h[t] = gp[t];
+          else
+            gp[t] = h[t];
+        }
+    }
+  }
+}
+
+template <int BN>
+__device__ __forceinline__ void apply_tile_transposed(const Epilogue& e, uint8_t* box, uint32_t tbase, int l, int row0w,
+                                                      int col0, int M, int N, int lane, int half) {
+  float alpha = e.alpha, beta = e.beta;
+  if (e.alpha_vec) alpha *= e.alpha_vec[l];
+  if (e.beta_vec) beta *= e.beta_vec[l];
+  __nv_bfloat16* W = static_cast<__nv_bfloat16*>(e.W[l]);
+  const bool vec = ((reinterpret_cast<uintptr_t>(W) & 15) == 0) && ((e.ldw & 7) == 0);
+  const int row = row0w + lane;
+  constexpr int NCH = BN / CH;
+  constexpr int STRIDE = EPI_WARPS / 4;
+#pragma unroll 1
+  for (int i = half; i < NCH; i += STRIDE) {
+    const int col = col0 + i * CH;
+    float v[32];
+    tmem_ld_32cols(tbase + i * CH, v);  // warp-collective
+    if (col >= N || row0w >= M) continue;
+    const int nrows = N - col < 32 ? N - col : 32;     // W rows of the box
+    const int ncols = M - row0w < 32 ? M - row0w : 32;  // W columns of the box
+    box_rw(box, W, e.ldw, col, row0w, nrows, ncols, vec, true, lane);
+    __syncwarp();
+    if (row < M) {
+      __nv_bfloat16* bx = reinterpret_cast<__nv_bfloat16*>(box);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (j >= nrows) break;
+        float o = alpha * v[j];
+        if (e.C != nullptr && beta != 0.f)
+          o += beta * load_elem(e.C, static_cast<long long>(l) * e.sc + static_cast<long long>(row) * e.ldc + col + j,
+                                e.c_f32);
+        if (e.diag != 0.f && col + j == row) o += e.diag;
+        const float w = __bfloat162float(bx[j * 32 + lane]);
+        bx[j * 32 + lane] = __float2bfloat16_rn(e.decay * w - e.lr_scale * o);
+      }
+    }
+    __syncwarp();
+    box_rw(box, W, e.ldw, col, row0w, nrows, ncols, vec, false, lane);
+    __syncwarp();  // the box is free for the next chunk
   }
 }
 
@@ -342,6 +440,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint32_t acc_phase = 0;
     StageState st;
     uint8_t* wstg = stg + ep * WARP_STG;
+    const bool apply_t = !staged && epi.mode == EPI_APPLY && epi.transposed && !epi.w_f32;
     for (long long t = blockIdx.x; t < total; t += gridDim.x) {
       int l, tm, tn;
       bool mir;
@@ -356,6 +455,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (staged) {
         store_tile_staged<BN>(epi, &tmC, &tmD, &tmDm, wstg, cbar + ep * NRING, tbase, l, tm * BM + ew * 32, tn * BN,
                               M, N, mir, lane, half, st, abort);
+      } else if (apply_t) {
+        apply_tile_transposed<BN>(epi, wstg, tbase, l, tm * BM + ew * 32, tn * BN, M, N, lane, half);
       } else {
 #pragma unroll 1
         for (int c0 = half * 32; c0 < BN; c0 += 32 * (EPI_WARPS / 4)) {
@@ -537,6 +638,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     uint32_t acc_phase = 0;
     StageState st;
     uint8_t* wstg = stg + ep * WARP_STG;
+    const bool apply_t = !staged && epi.mode == EPI_APPLY && epi.transposed && !epi.w_f32;
     for (long long t = pair; t < total; t += npairs) {
       int l, tm, tn;
       bool mir;
@@ -550,6 +652,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       if (staged) {
         store_tile_staged<P_BN>(epi, &tmC, &tmD, &tmDm, wstg, cbar + ep * NRING, tbase, l, row0 + ew * 32,
                                 tn * P_BN, M, N, mir, lane, half, st, abort);
+      } else if (apply_t) {
+        apply_tile_transposed<P_BN>(epi, wstg, tbase, l, row0 + ew * 32, tn * P_BN, M, N, lane, half);
       } else {
 #pragma unroll 1
         for (int c0 = half * 32; c0 < P_BN; c0 += 32 * (EPI_WARPS / 4)) {

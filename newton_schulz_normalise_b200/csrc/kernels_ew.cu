@@ -200,6 +200,86 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_tall_kernel(const Momentu
   if (threadIdx.x == 0) a.partials[static_cast<long long>(l) * a.nblk + blockIdx.x] = tot;
 }
 
+// Tall matrices, vector path (cols % 4 == 0, 16-byte aligned G and B):
+// 64 x 128 tiles.  Each warp reads 8 rows of the tile, a lane four
+// consecutive columns (one 16-byte load of B, one 8- or 16-byte load of G);
+// U goes to shared memory transposed, and each warp then writes rows of X
+// (stored columns) two elements per lane.  The shared tile is [128][64]
+// floats with the row index XOR-swizzled by an even key of the column, so
+// the transposed writes meet at most two lanes per bank and the 8-byte
+// reads of the write phase none.
+constexpr int TVR = 64, TVC = 128;
+__device__ __forceinline__ int tv_idx(int c, int r) { return c * TVR + (r ^ (((c >> 2) & 15) << 1)); }
+
+__global__ void __launch_bounds__(EW_THREADS) momentum_tall_vec_kernel(const MomentumArgs a) {
+  __shared__ __align__(16) float tile[TVC * TVR];
+  __shared__ float red[EW_THREADS / 32];
+  const int l = blockIdx.y;
+  const void* G = a.G[l];
+  float* B = static_cast<float*>(a.B[l]);
+  const long long xoff = static_cast<long long>(l) * a.cols * a.ldx;  // X is cols x rows, row stride ldx
+  const int tr = (a.rows + TVR - 1) / TVR, tc = (a.cols + TVC - 1) / TVC;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;  // 32 x 8
+  const float mu = a.mu;
+  float ss = 0.f;
+  for (int t = blockIdx.x; t < tr * tc; t += gridDim.x) {
+    const int r0 = (t / tc) * TVR, c0 = (t % tc) * TVC;
+    const int c = c0 + 4 * lane;  // this lane's four stored columns
+#pragma unroll 4
+    for (int k = 0; k < TVR / 8; ++k) {
+      const int rr = w + 8 * k;
+      const int r = r0 + rr;
+      float u[4] = {0.f, 0.f, 0.f, 0.f};
+      if (r < a.rows && c < a.cols) {  // cols % 4 == 0: the four columns are in range together
+        const long long i = static_cast<long long>(r) * a.cols + c;
+        float g[4];
+        if (a.g_f32) {
+          const float4 gv = __ldcs(reinterpret_cast<const float4*>(static_cast<const float*>(G) + i));
+          g[0] = gv.x; g[1] = gv.y; g[2] = gv.z; g[3] = gv.w;
+        } else {
+          const uint2 gv = __ldcs(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(G) + i));
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&gv);
+          const float2 g01 = __bfloat1622float2(h[0]), g23 = __bfloat1622float2(h[1]);
+          g[0] = g01.x; g[1] = g01.y; g[2] = g23.x; g[3] = g23.y;
+        }
+        const float4 bv = __ldcs(reinterpret_cast<const float4*>(B + i));
+        float b[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          b[j] = fmaf(mu, b[j], g[j]);
+          u[j] = a.nesterov ? fmaf(mu, b[j], g[j]) : b[j];
+          ss = fmaf(u[j], u[j], ss);
+        }
+        __stcs(reinterpret_cast<float4*>(B + i), make_float4(b[0], b[1], b[2], b[3]));
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tile[tv_idx(4 * lane + j, rr)] = u[j];
+    }
+    __syncthreads();
+    // X rows c0..c0+127 (stored columns), columns r0..r0+63: lane takes two
+#pragma unroll 4
+    for (int k = 0; k < TVC / 8; ++k) {
+      const int cc = w + 8 * k;
+      const int xr = c0 + cc, xc = r0 + 2 * lane;
+      const float2 v = *reinterpret_cast<const float2*>(&tile[tv_idx(cc, 2 * lane)]);
+      if (xr < a.cols && xc < a.rows) {
+        const long long o = xoff + static_cast<long long>(xr) * a.ldx + xc;
+        if (xc + 1 < a.rows) {
+          if (a.x_f32)
+            *reinterpret_cast<float2*>(static_cast<float*>(a.X) + o) = v;
+          else
+            *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(a.X) + o) = __floats2bfloat162_rn(v.x, v.y);
+        } else {
+          store_elem(a.X, o, v.x, a.x_f32);
+        }
+      }
+    }
+    __syncthreads();
+  }
+  const float tot = block_sum(ss, red);
+  if (threadIdx.x == 0) a.partials[static_cast<long long>(l) * a.nblk + blockIdx.x] = tot;
+}
+
 __global__ void norm_finalize_kernel(const float* __restrict__ partials, int nblk, float eps, float* s, float* s2) {
   const int l = blockIdx.x;
   __shared__ double red[32];
@@ -465,7 +545,13 @@ cudaError_t launch_momentum(const MomentumArgs& a, cudaStream_t s) {
   if (a.cnt > 65535) return cudaErrorInvalidValue;
   dim3 grid(a.nblk, a.cnt);
   if (a.transposed) {
-    momentum_tall_kernel<<<grid, EW_THREADS, 0, s>>>(a);
+    // the vector path reads four columns with one load: cols % 4 == 0 and
+    // 16-byte aligned G/B bases (a.aligned); X rows start 8-byte aligned
+    // (ldx % 8 == 0) for its two-element stores
+    if (a.cols % 4 == 0 && a.aligned && (a.ldx & 7) == 0)
+      momentum_tall_vec_kernel<<<grid, EW_THREADS, 0, s>>>(a);
+    else
+      momentum_tall_kernel<<<grid, EW_THREADS, 0, s>>>(a);
   } else {
     // The vector path needs cols % 8 == 0 (then ldx == cols) and 16-byte
     // aligned G/B bases (checked by the host: a.aligned).

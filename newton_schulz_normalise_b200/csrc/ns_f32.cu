@@ -102,6 +102,77 @@ __device__ __forceinline__ void sym_tile(int u, int T, int& tm, int& tn) {
   tn = tm + u;
 }
 
+// Loads the float4 at element k (of kc valid) of a row, zero past the end.
+__device__ __forceinline__ float4 ld_row4(const float* src, int k, int kc) {
+  if (k + 4 <= kc) return *reinterpret_cast<const float4*>(src);
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (k < kc) v.x = src[0];
+  if (k + 1 < kc) v.y = src[1];
+  if (k + 2 < kc) v.z = src[2];
+  return v;
+}
+
+constexpr int LB = 8;  // float4 loads per thread in flight before they are stored
+
+// Stages a 16-row x kc slab whose rows are contiguous along k (rows beyond
+// `rows` read as zero) into dst[r * F_LD + k], LB loads in flight per thread.
+__device__ __forceinline__ void stage_rows(float* dst, const float* __restrict__ src, long long ld, int r0, int rows,
+                                           int k0, int kc) {
+  const int kq = (kc + 3) / 4;  // float4 per row
+  const int total = FT * kq;
+  for (int base = threadIdx.x; base < total; base += F_THREADS * LB) {
+    float4 v[LB];
+#pragma unroll
+    for (int j = 0; j < LB; ++j) {
+      const int i = base + j * F_THREADS;
+      v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < total) {
+        const int r = i / kq, k = (i % kq) * 4;
+        if (r0 + r < rows) v[j] = ld_row4(src + static_cast<long long>(r0 + r) * ld + k0 + k, k, kc);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < LB; ++j) {
+      const int i = base + j * F_THREADS;
+      if (i < total) {
+        const int r = i / kq, k = (i % kq) * 4;
+        *reinterpret_cast<float4*>(dst + r * F_LD + k) = v[j];
+      }
+    }
+  }
+}
+
+// Stages kc rows of 16 columns (k-major storage: row k, columns c0..c0+15)
+// transposed into dst[c * F_LD + k]; columns beyond `cols` and rows from kc
+// up to the next multiple of 4 (the compute loop's padding) are zero.
+__device__ __forceinline__ void stage_cols(float* dst, const float* __restrict__ src, long long ld, int c0, int cols,
+                                           int k0, int kc) {
+  const int total = ((kc + 3) & ~3) * (FT / 4);
+  for (int base = threadIdx.x; base < total; base += F_THREADS * LB) {
+    float4 v[LB];
+#pragma unroll
+    for (int j = 0; j < LB; ++j) {
+      const int i = base + j * F_THREADS;
+      v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < total) {
+        const int k = i / (FT / 4), cc = (i % (FT / 4)) * 4;
+        if (k < kc) v[j] = ld_row4(src + static_cast<long long>(k0 + k) * ld + c0 + cc, c0 + cc, cols);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < LB; ++j) {
+      const int i = base + j * F_THREADS;
+      if (i < total) {
+        const int k = i / (FT / 4), cc = (i % (FT / 4)) * 4;
+        dst[(cc + 0) * F_LD + k] = v[j].x;
+        dst[(cc + 1) * F_LD + k] = v[j].y;
+        dst[(cc + 2) * F_LD + k] = v[j].z;
+        dst[(cc + 3) * F_LD + k] = v[j].w;
+      }
+    }
+  }
+}
+
 // One 16 x 16 output tile: out(ty, tx) = sum_k Aop[r0 + ty][k] * B(k, c0 + tx),
 // B(k, c) = Bop[c][k] (b_kmajor) or Bop[k][c].  Rows of Aop / Bop beyond their
 // extents read as zero.  Returns this thread's sum.
@@ -114,58 +185,11 @@ __device__ float tile_dot(const float* __restrict__ Aop, long long lda, int arow
     const int kc = min(FKC, K - k0);
     const int kc4 = (kc + 3) & ~3;
     __syncthreads();  // the previous chunk's (or tile's) reads of As / Bs are done
-    // A slab: 16 rows x kc, float4 along k (rows 16-byte aligned: ld % 8 == 0)
-    for (int i = tid; i < FT * (kc4 / 4); i += F_THREADS) {
-      const int r = i / (kc4 / 4), k = (i % (kc4 / 4)) * 4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r0 + r < arows) {
-        const float* src = Aop + static_cast<long long>(r0 + r) * lda + k0 + k;
-        if (k + 4 <= kc) {
-          v = *reinterpret_cast<const float4*>(src);
-        } else {
-          v.x = k < kc ? src[0] : 0.f;
-          v.y = k + 1 < kc ? src[1] : 0.f;
-          v.z = k + 2 < kc ? src[2] : 0.f;
-        }
-      }
-      *reinterpret_cast<float4*>(As + r * F_LD + k) = v;
-    }
-    if (b_kmajor) {  // B slab rows = output columns, contiguous along k
-      for (int i = tid; i < FT * (kc4 / 4); i += F_THREADS) {
-        const int cc = i / (kc4 / 4), k = (i % (kc4 / 4)) * 4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (c0 + cc < bcols) {
-          const float* src = Bop + static_cast<long long>(c0 + cc) * ldb + k0 + k;
-          if (k + 4 <= kc) {
-            v = *reinterpret_cast<const float4*>(src);
-          } else {
-            v.x = k < kc ? src[0] : 0.f;
-            v.y = k + 1 < kc ? src[1] : 0.f;
-            v.z = k + 2 < kc ? src[2] : 0.f;
-          }
-        }
-        *reinterpret_cast<float4*>(Bs + cc * F_LD + k) = v;
-      }
-    } else {  // B stored k-major rows of columns: read 4 columns at a time, store transposed
-      for (int i = tid; i < kc4 * (FT / 4); i += F_THREADS) {
-        const int k = i / (FT / 4), cc = (i % (FT / 4)) * 4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (k < kc) {
-          const float* src = Bop + static_cast<long long>(k0 + k) * ldb + c0 + cc;
-          if (c0 + cc + 4 <= bcols) {
-            v = *reinterpret_cast<const float4*>(src);
-          } else {
-            v.x = c0 + cc < bcols ? src[0] : 0.f;
-            v.y = c0 + cc + 1 < bcols ? src[1] : 0.f;
-            v.z = c0 + cc + 2 < bcols ? src[2] : 0.f;
-          }
-        }
-        Bs[(cc + 0) * F_LD + k] = v.x;
-        Bs[(cc + 1) * F_LD + k] = v.y;
-        Bs[(cc + 2) * F_LD + k] = v.z;
-        Bs[(cc + 3) * F_LD + k] = v.w;
-      }
-    }
+    stage_rows(As, Aop, lda, r0, arows, k0, kc);
+    if (b_kmajor)
+      stage_rows(Bs, Bop, ldb, c0, bcols, k0, kc);
+    else
+      stage_cols(Bs, Bop, ldb, c0, bcols, k0, kc);
     __syncthreads();
     const float* a = As + ty * F_LD;
     const float* b = Bs + tx * F_LD;

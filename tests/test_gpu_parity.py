@@ -313,3 +313,19 @@ def test_resident_medium_nonfinite_stays_in_its_matrix(dmuon_lib):
     for i in (0, 2):
         _, Oo = oracle_update(Gs[i], Ms[i])
         assert rel_fro(to64(Os[i]), Oo) <= BF16_TOL, i
+
+
+@pytest.mark.parametrize("pdt", ["bf16", "f32"])
+def test_tall_momentum_vector_path(dmuon_lib, pdt):
+    """Tall matrices whose column count is a multiple of 4 take the vector
+    momentum kernel (64 x 128 tiles, transposed through shared memory): odd
+    and ragged row counts, a partial last column tile, and an aligned one."""
+    shapes = [(301, 100), (257, 36), (130, 64), (1031, 260)]
+    std = 0.02 if pdt == "f32" else 1e-3
+    Ws, Gs, Ms = make_inputs(shapes, seed=96, pdt=pdt, m_std=std, g_std=std)
+    Os, Bn = gpu_update(dmuon_lib, Gs, Ms)
+    tol = F32_TOL if pdt == "f32" else BF16_TOL
+    for i in range(len(shapes)):
+        check_momentum(Bn[i], Gs[i], Ms[i], 0.95)
+        _, Oo = oracle_update(Gs[i], Ms[i])
+        assert rel_fro(to64(Os[i]), Oo) <= tol, (shapes[i], rel_fro(to64(Os[i]), Oo))
