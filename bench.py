@@ -369,6 +369,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--variant", default="auto", choices=["auto", "direct", "gram", "batched"],
+                    help="Newton-Schulz form for every shape group (default: the autotuner's choice)")
     ap.add_argument("--step-only", action="store_true",
                     help="time the step alone: no per-kernel pass, end-to-end, AdamW or CPU baseline "
                          "(profiler runs)")
@@ -401,7 +403,7 @@ def main():
     Ws, Gs, Ms = wl.generate(w, device=dev)
     shapes = w.shapes()
     pdt = B.DMUON_BF16 if w.param_dtype == "bf16" else B.DMUON_F32
-    opts = B.options(pdt, pdt)
+    opts = B.options(pdt, pdt, variant=args.variant)
     # the parameter lists are marshalled once, as an optimiser loop would
     tW, tG, tM = B.TensorList(Ws), B.TensorList(Gs), B.TensorList(Ms)
 
@@ -539,7 +541,8 @@ def main():
     simt = kinds[B.KIND_SIMT_GEMM]
     # executed NS FLOPs per step (symmetric products count their computed tiles only)
     flops = (gemm["flops"] + simt["flops"]) / kt_steps
-    dense = sum(ns_flops(r, c, w.ns_steps, variants.get((r, c), "direct")) for r, c in shapes)
+    # plans are keyed by the iterate's shape (min, max): a weight and its transpose share one
+    dense = sum(ns_flops(r, c, w.ns_steps, variants.get((min(r, c), max(r, c)), "direct")) for r, c in shapes)
     tflops = flops / (ms_per_step * 1e-3) / 1e12
     peak_tc = peaks["bf16_tflops"]
     peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])

@@ -376,9 +376,13 @@ struct Hyper {
   int steps, nesterov;
 };
 
+// A chunk of a shape group.  Its geometry g is the iterate's (m x n, m <= n):
+// the first nwide matrices are stored m x n, the others n x m (the transposed
+// weights of the same dimensions), and the Newton-Schulz products serve both.
 struct Chunk {
   const Geo* g;
   int cnt;
+  int nwide;
   uint8_t* base;  // scratch of this chunk
   Layout L;
   void* const* Gt;  // device pointer tables for this chunk
@@ -431,29 +435,36 @@ Epilogue store_epi(void* D, long long ldd, long long sd, bool f32, float alpha, 
   return e;
 }
 
-// Runs K1 (momentum + norm partials) and the finalize for a chunk.
+// Runs K1 (momentum + norm partials) for each orientation part of a chunk
+// (every launch covers ch.nblk partial slots per matrix), then the finalize.
 int run_momentum(const Chunk& ch, bool f32, bool g_f32, const Hyper& h, cudaStream_t s) {
   const Geo& g = *ch.g;
-  MomentumArgs a{};
-  a.G = ch.Gt;
-  a.B = ch.Bt;
-  a.X = at<void>(ch, ch.L.X0);
-  a.ldx = g.ldx;
-  a.x_f32 = f32;
-  a.g_f32 = g_f32;
-  a.rows = g.rows;
-  a.cols = g.cols;
-  a.transposed = g.transposed;
-  a.cnt = ch.cnt;
-  a.mu = h.mu;
-  a.nesterov = h.nesterov;
-  a.partials = at<float>(ch, ch.L.partials);
-  a.nblk = ch.nblk;
-  a.aligned = ch.aligned;
-  const double bytes = static_cast<double>(g.rows) * g.cols * ch.cnt * ((g_f32 ? 4 : 2) + 8 + (f32 ? 4 : 2));
-  cudaError_t e = launch_k(KIND_EW, 0.0, bytes, s, [&] { return launch_momentum(a, s); });
-  if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "momentum kernel: %s", cudaGetErrorString(e));
-  e = launch_k(KIND_OTHER, 0.0, 0.0, s, [&] {
+  auto part = [&](int off, int cnt, bool tall) -> int {
+    MomentumArgs a{};
+    a.G = ch.Gt + off;
+    a.B = ch.Bt + off;
+    a.X = at<uint8_t>(ch, ch.L.X0) + static_cast<size_t>(off) * g.x_elems() * g.esz;
+    a.ldx = g.ldx;
+    a.x_f32 = f32;
+    a.g_f32 = g_f32;
+    a.rows = tall ? g.n : g.m;
+    a.cols = tall ? g.m : g.n;
+    a.transposed = tall ? 1 : 0;
+    a.cnt = cnt;
+    a.mu = h.mu;
+    a.nesterov = h.nesterov;
+    a.partials = at<float>(ch, ch.L.partials) + static_cast<size_t>(off) * ch.nblk;
+    a.nblk = ch.nblk;
+    a.aligned = ch.aligned;
+    const double bytes = static_cast<double>(g.m) * g.n * cnt * ((g_f32 ? 4 : 2) + 8 + (f32 ? 4 : 2));
+    cudaError_t e = launch_k(KIND_EW, 0.0, bytes, s, [&] { return launch_momentum(a, s); });
+    if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "momentum kernel: %s", cudaGetErrorString(e));
+    return DMUON_OK;
+  };
+  int rc;
+  if (ch.nwide > 0 && (rc = part(0, ch.nwide, false))) return rc;
+  if (ch.cnt > ch.nwide && (rc = part(ch.nwide, ch.cnt - ch.nwide, true))) return rc;
+  cudaError_t e = launch_k(KIND_OTHER, 0.0, 0.0, s, [&] {
     return launch_norm_finalize(at<float>(ch, ch.L.partials), ch.nblk, ch.cnt, h.eps, at<float>(ch, ch.L.s),
                                 at<float>(ch, ch.L.s2), s);
   });
@@ -461,61 +472,115 @@ int run_momentum(const Chunk& ch, bool f32, bool g_f32, const Hyper& h, cudaStre
   return DMUON_OK;
 }
 
+// Partial-sum slots per matrix for a chunk holding wide and/or tall
+// matrices of the iterate geometry g (the larger of the two launches' grids).
+int chunk_nblk(const Geo& g, bool wide, bool tall) {
+  int nb = 1;
+  if (wide) nb = std::max(nb, momentum_partials(g.m, g.n));
+  if (tall) nb = std::max(nb, momentum_partials(g.n, g.m));
+  return nb;
+}
+
+// The epilogue e for the matrices off, off+1, ... of its tables.
+Epilogue shift_epi(Epilogue e, int off) {
+  if (e.W) e.W += off;
+  if (e.Out) e.Out += off;
+  if (e.alpha_vec) e.alpha_vec += off;
+  if (e.beta_vec) e.beta_vec += off;
+  if (e.D) e.D = static_cast<uint8_t*>(e.D) + static_cast<size_t>(off) * e.sd * (e.d_f32 ? 4 : 2);
+  return e;
+}
+
 // Newton-Schulz on X0 (unnormalised U, scale s folded into the first
-// products), finishing with `fin` (apply / out / store) on the result.  Its
-// launches are timed as one chain.
-int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const Hyper& h, const Epilogue& fin_in,
-           int cnt, cudaStream_t s) {
+// products), finishing with an epilogue (apply / out / store) on the result:
+// fin_w for the chunk's first ch.nwide matrices (stored m x n), fin_t for the
+// rest (stored n x m).  Every product but the last serves both orientations
+// in one launch; the last runs once per orientation present.  Kernels that
+// run every step in one launch (and the zero-step scale) run once per
+// orientation part.  The launches are timed as one chain.
+int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const Hyper& h, const Epilogue& fin_w,
+           const Epilogue& fin_t, int cnt, cudaStream_t s) {
   const Geo& g = *ch.g;
   const int m = g.m, n = g.n;
   const long long sx = g.x_elems(), sq = g.q_elems();
   const float* sv = at<float>(ch, ch.L.s);
   const float* s2v = at<float>(ch, ch.L.s2);
-  void* X0 = at<void>(ch, ch.L.X0);
-  Epilogue fin = fin_in;
+  uint8_t* X0 = at<uint8_t>(ch, ch.L.X0);
+  const int split = std::min(std::max(ch.nwide, 0), cnt);
+  auto xoff = [&](int off) { return X0 + static_cast<size_t>(off) * sx * g.esz; };
+  // runs one(off, count, epilogue) for each orientation part present
+  auto parts = [&](auto&& one) -> int {
+    int r = DMUON_OK;
+    if (split > 0 && (r = one(0, split, shift_epi(fin_w, 0)))) return r;
+    if (cnt > split) r = one(split, cnt - split, shift_epi(fin_t, split));
+    return r;
+  };
   int rc;
   TimedChain chain(s, !f32 && variant != DMUON_VARIANT_BATCHED && tile == 512 && h.steps > 0);
   if (h.steps == 0) {  // O = X0 = s U; the kernel folds s in
-    fin.alpha = 1.f;
-    fin.alpha_vec = nullptr;
-    fin.beta = 0.f;
-    fin.C = nullptr;
-    cudaError_t e = launch_k(KIND_OTHER, 0.0, 0.0, s, [&] {
-      return launch_scale_epilogue(X0, g.ldx, f32, m, n, cnt, sv, fin, s);
+    return parts([&](int off, int nn, Epilogue fin) -> int {
+      fin.alpha = 1.f;
+      fin.alpha_vec = nullptr;
+      fin.beta = 0.f;
+      fin.C = nullptr;
+      cudaError_t e = launch_k(KIND_OTHER, 0.0, 0.0, s, [&] {
+        return launch_scale_epilogue(xoff(off), g.ldx, f32, m, n, nn, sv + off, fin, s);
+      });
+      if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "scale epilogue: %s", cudaGetErrorString(e));
+      return DMUON_OK;
     });
-    if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "scale epilogue: %s", cudaGetErrorString(e));
-    return DMUON_OK;
   }
   if (variant == DMUON_VARIANT_BATCHED && f32) {  // fp32: every step in one cooperative launch
-    NsF32 a{static_cast<const float*>(X0), at<float>(ch, ch.L.Xp), at<float>(ch, ch.L.Xq), at<float>(ch, ch.L.A),
-            at<float>(ch, ch.L.Bm), g.ldx, g.ldm, sx, sq, sv, s2v, cnt, m, n, h.steps, h.a, h.b, h.c, fin,
-            at<unsigned>(ch, ch.L.sync)};
-    const double T = (m + 15) / 16;
-    const double symf = (T * (T + 1) / 2) / (T * T);
-    const double fl = 2.0 * h.steps * cnt * (symf * m * static_cast<double>(m) * n + symf * m * static_cast<double>(m) * m +
-                                            m * static_cast<double>(m) * n);
-    cudaError_t e = launch_k(KIND_SIMT_GEMM, fl, 0.0, s, [&] { return launch_ns_f32(a, s, c.err_dev, c.num_sms); });
-    if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "fp32 resident kernel: %s", cudaGetErrorString(e));
-    return DMUON_OK;
+    return parts([&](int off, int nn, Epilogue fin) -> int {
+      NsF32 a{reinterpret_cast<const float*>(xoff(off)), at<float>(ch, ch.L.Xp), at<float>(ch, ch.L.Xq),
+              at<float>(ch, ch.L.A), at<float>(ch, ch.L.Bm), g.ldx, g.ldm, sx, sq, sv + off, s2v + off, nn, m, n,
+              h.steps, h.a, h.b, h.c, fin, at<unsigned>(ch, ch.L.sync)};
+      const double T = (m + 31) / 32;
+      const double symf = (T * (T + 1) / 2) / (T * T);
+      const double fl = 2.0 * h.steps * nn *
+                        (symf * m * static_cast<double>(m) * n + symf * m * static_cast<double>(m) * m +
+                         m * static_cast<double>(m) * n);
+      cudaError_t e = launch_k(KIND_SIMT_GEMM, fl, 0.0, s, [&] { return launch_ns_f32(a, s, c.err_dev, c.num_sms); });
+      if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "fp32 resident kernel: %s", cudaGetErrorString(e));
+      return DMUON_OK;
+    });
   }
   if (variant == DMUON_VARIANT_BATCHED && !ns_small_supported(m, n)) {  // bf16, medium: one CTA pair per matrix
-    cudaError_t e = launch_k(KIND_TC_GEMM, ns_mid_flops(m, n, h.steps, cnt), 0.0, s, [&] {
-      return launch_ns_mid(X0, at<void>(ch, ch.L.Xp), g.ldx, sv, s2v, cnt, m, n, h.steps, h.a, h.b, h.c, fin, s,
-                           c.err_dev, c.num_sms);
+    return parts([&](int off, int nn, Epilogue fin) -> int {
+      cudaError_t e = launch_k(KIND_TC_GEMM, ns_mid_flops(m, n, h.steps, nn), 0.0, s, [&] {
+        return launch_ns_mid(xoff(off), at<void>(ch, ch.L.Xp), g.ldx, sv + off, s2v + off, nn, m, n, h.steps, h.a,
+                             h.b, h.c, fin, s, c.err_dev, c.num_sms);
+      });
+      if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "resident medium-matrix kernel: %s", cudaGetErrorString(e));
+      return DMUON_OK;
     });
-    if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "resident medium-matrix kernel: %s", cudaGetErrorString(e));
-    return DMUON_OK;
   }
   if (variant == DMUON_VARIANT_BATCHED) {  // resident small-matrix kernel (bf16)
-    cudaError_t e = launch_k(KIND_TC_GEMM, 2.0 * h.steps * (2.0 * 128 * 128 * g.n + 2.0 * 128 * 128 * 128) *
-                                               ((cnt + ns_small_group(m) - 1) / ns_small_group(m)),
-                             0.0, s, [&] {
-                               return launch_ns_small(X0, g.ldx, sv, s2v, cnt, m, n, h.steps, h.a, h.b, h.c, fin, s,
-                                                      c.err_dev);
-                             });
-    if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "resident small-matrix kernel: %s", cudaGetErrorString(e));
-    return DMUON_OK;
+    return parts([&](int off, int nn, Epilogue fin) -> int {
+      cudaError_t e = launch_k(KIND_TC_GEMM, 2.0 * h.steps * (2.0 * 128 * 128 * g.n + 2.0 * 128 * 128 * 128) *
+                                                 ((nn + ns_small_group(m) - 1) / ns_small_group(m)),
+                               0.0, s, [&] {
+                                 return launch_ns_small(xoff(off), g.ldx, sv + off, s2v + off, nn, m, n, h.steps, h.a,
+                                                        h.b, h.c, fin, s, c.err_dev);
+                               });
+      if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "resident small-matrix kernel: %s", cudaGetErrorString(e));
+      return DMUON_OK;
+    });
   }
+  // The last product O = scale * Aop Bx (m x n, K = m, Bx the MN-major iterate),
+  // once per orientation part with its epilogue.
+  auto final_product = [&](const void* Aop, const void* Bx, bool scale) -> int {
+    return parts([&](int off, int nn, Epilogue fin) -> int {
+      fin.alpha = 1.f;
+      fin.alpha_vec = scale ? sv + off : nullptr;
+      fin.beta = 0.f;
+      fin.beta_vec = nullptr;
+      fin.C = nullptr;
+      return gemm(c, nn, f32, tile, false, static_cast<const uint8_t*>(Aop) + static_cast<size_t>(off) * sq * g.esz,
+                  g.ldm, sq, static_cast<const uint8_t*>(Bx) + static_cast<size_t>(off) * sx * g.esz, g.ldx, sx, false,
+                  m, n, m, fin, s);
+    });
+  };
   if (variant == DMUON_VARIANT_GRAM) {
     // Every m x m product takes its right operand as stored (MN-major B), not
     // as the transpose of a matrix that is symmetric only up to rounding:
@@ -557,11 +622,7 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
       }
     }
     // O = s * Q_K U
-    fin.alpha = 1.f;
-    fin.alpha_vec = sv;
-    fin.beta = 0.f;
-    fin.C = nullptr;
-    return gemm(c, cnt, f32, tile, false, Q[qi], g.ldm, sq, X0, g.ldx, sx, false, m, n, m, fin, s);
+    return final_product(Q[qi], X0, true);
   }
   // ---------------- direct form
   // Per step: A = X X^T, P = c A^2 + b A + a I, X' = P X.  Folding a X into
@@ -589,14 +650,10 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
     rc = gemm(c, cnt, f32, tile, true, A, g.ldm, sq, A, g.ldm, sq, false, m, m, m, ep, s);
     if (rc) return rc;
     // X' = P X   (times s on the first step)
+    if (last) return final_product(P, cur, first);
     void* nxt = bufs[k & 1];
-    Epilogue eu = last ? fin : store_epi(nxt, g.ldx, sx, f32, 1.f, nullptr);
-    eu.alpha = 1.f;
-    eu.alpha_vec = first ? sv : nullptr;
-    eu.beta = 0.f;
-    eu.beta_vec = nullptr;
-    eu.C = nullptr;
-    rc = gemm(c, cnt, f32, tile, false, P, g.ldm, sq, cur, g.ldx, sx, false, m, n, m, eu, s);
+    rc = gemm(c, cnt, f32, tile, false, P, g.ldm, sq, cur, g.ldx, sx, false, m, n, m,
+              store_epi(nxt, g.ldx, sx, f32, 1.f, first ? sv : nullptr), s);
     if (rc) return rc;
     cur = nxt;
   }
@@ -604,11 +661,16 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
 }
 
 // ------------------------------------------------------------------ step
+// A shape group: the matrices whose iterate is m x n (rows = m <= cols = n),
+// whether stored m x n or n x m (a weight and a transposed weight of the
+// same dimensions share every Newton-Schulz product).  idx lists the ones
+// stored m x n first, then the ntall stored n x m.
 struct Group {
   long long rows, cols;
   std::vector<int> idx;
   Plan plan;
   int chunk;
+  int ntall;
 };
 
 struct Request {
@@ -698,10 +760,12 @@ int upload_tables(DeviceCtx& c, const std::vector<void*>& host, void* dev, cudaS
   return DMUON_OK;
 }
 
-Epilogue final_epilogue(const Request& r, const Geo& g, const Chunk& ch, bool f32) {
+// The last product's epilogue for the chunk's matrices stored m x n
+// (tall = false) or n x m (tall = true; the update is written transposed).
+Epilogue final_epilogue(const Request& r, const Geo& g, const Chunk& ch, bool f32, bool tall) {
   Epilogue e{};
-  e.transposed = g.transposed;
-  e.ldw = g.cols;
+  e.transposed = tall ? 1 : 0;
+  e.ldw = tall ? g.m : g.n;
   e.w_f32 = f32;
   if (r.out) {
     e.mode = EPI_OUT;
@@ -718,7 +782,7 @@ Epilogue final_epilogue(const Request& r, const Geo& g, const Chunk& ch, bool f3
 int time_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const Hyper& h, const Epilogue& fin,
             int cnt, cudaStream_t s, float* ms) {
   CUDA_TRY(cudaEventRecord(c.tune_a, s));
-  int rc = run_ns(c, ch, f32, variant, tile, h, fin, cnt, s);
+  int rc = run_ns(c, ch, f32, variant, tile, h, fin, fin, cnt, s);
   if (rc) return rc;
   CUDA_TRY(cudaEventRecord(c.tune_b, s));
   CUDA_TRY(cudaEventSynchronize(c.tune_b));
@@ -781,7 +845,7 @@ int autotune(DeviceCtx& c, const Chunk& ch, bool f32, const Hyper& h, int forced
     Epilogue fin = store_epi(dst, g.ldx, g.x_elems(), f32, 1.f, nullptr);
     float ms = 0.f;
     // warm once (first launch of a kernel instance loads the module), then time
-    int rc = run_ns(c, ch, f32, v, tile, h, fin, probe, s);
+    int rc = run_ns(c, ch, f32, v, tile, h, fin, fin, probe, s);
     if (rc) return rc;
     rc = time_ns(c, ch, f32, v, tile, h, fin, probe, s, &ms);
     if (rc) return rc;
@@ -891,18 +955,25 @@ int run_step(Request& r) {
   const bool f32 = r.o.param_dtype == DMUON_F32;
   const bool g_f32 = r.o.grad_dtype == DMUON_F32;
 
-  // group by shape, in order of first appearance
+  // group by iterate shape (m, n), in order of first appearance; inside a
+  // group the matrices stored m x n come first
   std::vector<Group> groups;
   {
     std::map<std::pair<long long, long long>, int> gi;
     for (int i = 0; i < r.count; ++i) {
-      auto key = std::make_pair(static_cast<long long>(r.shapes[2 * i]), static_cast<long long>(r.shapes[2 * i + 1]));
+      const long long rr = r.shapes[2 * i], cc = r.shapes[2 * i + 1];
+      auto key = std::make_pair(std::min(rr, cc), std::max(rr, cc));
       auto it = gi.find(key);
       if (it == gi.end()) {
         it = gi.emplace(key, static_cast<int>(groups.size())).first;
-        groups.push_back(Group{key.first, key.second, {}, Plan{}, 0});
+        groups.push_back(Group{key.first, key.second, {}, Plan{}, 0, 0});
       }
       groups[it->second].idx.push_back(i);
+    }
+    for (Group& gr : groups) {
+      auto tall = [&](int i) { return r.shapes[2 * i] > r.shapes[2 * i + 1]; };
+      std::stable_partition(gr.idx.begin(), gr.idx.end(), [&](int i) { return !tall(i); });
+      gr.ntall = static_cast<int>(std::count_if(gr.idx.begin(), gr.idx.end(), tall));
     }
   }
   // plans: cache lookup; misses are tuned on this call's data below
@@ -930,7 +1001,7 @@ int run_step(Request& r) {
         miss[k] = true;
       }
     }
-    const int nblk = momentum_partials(geos[k].rows, geos[k].cols);
+    const int nblk = chunk_nblk(geos[k], gr.ntall < static_cast<int>(gr.idx.size()), gr.ntall > 0);
     Layout L = make_layout(geos[k], gr.chunk, nblk);
     size_t need = L.total;
     if (miss[k]) need += 2 * align256(static_cast<size_t>(gr.chunk) * geos[k].x_elems() * geos[k].esz) + 256;
@@ -1096,8 +1167,9 @@ int run_step(Request& r) {
       Chunk ch;
       ch.g = &g;
       ch.cnt = std::min(gr.chunk, total - c0);
+      ch.nwide = std::min(std::max(total - gr.ntall - c0, 0), ch.cnt);
       ch.base = ws + region_off[ln];
-      ch.nblk = momentum_partials(g.rows, g.cols);
+      ch.nblk = chunk_nblk(g, gr.ntall < total, gr.ntall > 0);
       ch.L = make_layout(g, gr.chunk, ch.nblk);
       const int p = gstart[k] + c0;
       ch.Gt = dtab + p;
@@ -1139,8 +1211,8 @@ int run_step(Request& r) {
         std::lock_guard<std::mutex> lk2(g_cache_mu);
         if (r.o.variant == DMUON_VARIANT_AUTO || !g_cache.count(key)) g_cache[key] = pl;
       }
-      Epilogue fin = final_epilogue(r, g, ch, f32);
-      rc = run_ns(c, ch, f32, gr.plan.variant, gr.plan.tile, r.h, fin, ch.cnt, gs);
+      rc = run_ns(c, ch, f32, gr.plan.variant, gr.plan.tile, r.h, final_epilogue(r, g, ch, f32, false),
+                  final_epilogue(r, g, ch, f32, true), ch.cnt, gs);
       if (rc) return rc;
       if (r.grads_host) {
         if (r.params_host) {  // copy-out: the chunk's updated parameters
@@ -1163,8 +1235,8 @@ int run_step(Request& r) {
       }
     }
     if (trace_on())
-      fprintf(stderr, "[dmuon] group %lldx%lld x%d: variant=%d tile=%d chunk=%d cost=%.3f ms stream=%d\n", gr.rows,
-              gr.cols, total, gr.plan.variant, gr.plan.tile, gr.chunk, gr.plan.cost_ms, lane[k]);
+      fprintf(stderr, "[dmuon] group %lldx%lld x%d (%d stored transposed): variant=%d tile=%d chunk=%d cost=%.3f ms stream=%d\n",
+              gr.rows, gr.cols, total, gr.ntall, gr.plan.variant, gr.plan.tile, gr.chunk, gr.plan.cost_ms, lane[k]);
   }
   if (forked) {
     for (int i = 0; i < DeviceCtx::kSide; ++i)
@@ -1313,7 +1385,8 @@ int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows,
   int rc = validate(r);
   if (rc) return rc;
   const bool f32 = o.param_dtype == DMUON_F32;
-  const Geo g = make_geo(rows, cols, f32);
+  const bool tall = rows > cols;
+  const Geo g = make_geo(std::min(rows, cols), std::max(rows, cols), f32);  // the iterate, m x n
   // plan: the resident kernel when it is asked for and the shape fits it;
   // else the plan the autotuner cached for this shape (count 1), else the
   // direct form (a forced variant the shape cannot take runs as AUTO)
@@ -1325,7 +1398,7 @@ int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows,
     const int want = o.variant == DMUON_VARIANT_BATCHED ? DMUON_VARIANT_AUTO : o.variant;
     if (want == DMUON_VARIANT_DIRECT || want == DMUON_VARIANT_GRAM) plan.variant = want;
     std::lock_guard<std::mutex> lk(g_cache_mu);
-    auto it = g_cache.find(Key{rows, cols, f32 ? 1 : 0, ns_steps, 1});
+    auto it = g_cache.find(Key{g.m, g.n, f32 ? 1 : 0, ns_steps, 1});
     if (it != g_cache.end() && (want == DMUON_VARIANT_AUTO || it->second.variant == want)) plan = it->second;
   }
   void* base = nullptr;
@@ -1334,7 +1407,7 @@ int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows,
   if (rc) return rc;
   int sms = 0;
   CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  const int nblk = momentum_partials(g.rows, g.cols);
+  const int nblk = chunk_nblk(g, !tall, tall);
   const Layout L = make_layout(g, 1, nblk);
   const size_t header = 256;  // 4 pointer slots and the device error word
   const size_t need = header + L.total;
@@ -1372,6 +1445,7 @@ int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows,
   Chunk ch;
   ch.g = &g;
   ch.cnt = 1;
+  ch.nwide = tall ? 0 : 1;
   ch.base = sb + header;
   ch.L = L;
   ch.Gt = dtab;
@@ -1385,10 +1459,10 @@ int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows,
   Epilogue fin{};
   fin.mode = EPI_OUT;
   fin.Out = ch.Ot;
-  fin.transposed = g.transposed;
-  fin.ldw = g.cols;
+  fin.transposed = tall ? 1 : 0;
+  fin.ldw = tall ? g.m : g.n;
   fin.w_f32 = f32;
-  rc = run_ns(c, ch, f32, plan.variant, plan.tile, r.h, fin, 1, s);
+  rc = run_ns(c, ch, f32, plan.variant, plan.tile, r.h, fin, fin, 1, s);
   if (rc) return rc;
   if (fault_wait()) {  // DMUON_FAULT=wait: a bounded wait that runs out, as a stalled pipeline would
     e = launch_wait_selftest(dev_err, 20000000ull, s);
@@ -1647,10 +1721,12 @@ int dmuon_workspace_size(const int64_t* shapes, int count, int param_dtype, size
   t_err.clear();
   if (!bytes || (count > 0 && !shapes) || count < 0) return fail(DMUON_ERR_INVALID, "bad arguments");
   const bool f32 = param_dtype == DMUON_F32;
-  std::map<std::pair<long long, long long>, int> counts;
+  std::map<std::pair<long long, long long>, std::pair<int, int>> counts;  // (m, n) -> (stored m x n, stored n x m)
   for (int i = 0; i < count; ++i) {
-    if (shapes[2 * i] <= 0 || shapes[2 * i + 1] <= 0) return fail(DMUON_ERR_INVALID, "bad shape");
-    counts[{shapes[2 * i], shapes[2 * i + 1]}]++;
+    const long long rr = shapes[2 * i], cc = shapes[2 * i + 1];
+    if (rr <= 0 || cc <= 0) return fail(DMUON_ERR_INVALID, "bad shape");
+    auto& e = counts[{std::min(rr, cc), std::max(rr, cc)}];
+    (rr > cc ? e.second : e.first)++;
   }
   // the first call runs every group on one stream (with autotune scratch);
   // later calls may give up to three small groups a region each
@@ -1661,12 +1737,13 @@ int dmuon_workspace_size(const int64_t* shapes, int count, int param_dtype, size
   cudaGetLastError();
   for (auto& kv : counts) {
     Geo g = make_geo(kv.first.first, kv.first.second, f32);
-    int ch = chunk_size(g, kv.second);
-    Layout L = make_layout(g, ch, momentum_partials(g.rows, g.cols));
+    const int total = kv.second.first + kv.second.second;
+    int ch = chunk_size(g, total);
+    Layout L = make_layout(g, ch, chunk_nblk(g, kv.second.first > 0, kv.second.second > 0));
     const size_t n_tune = align256(L.total + 2 * align256(static_cast<size_t>(ch) * g.x_elems() * g.esz) + 256);
     need = std::max(need, n_tune);
-    const bool maybe_small = !f32 && kv.second <= ch && (tc_gemm_tiles(g.m, g.n, ch, 128, false) < 2LL * sms ||
-                                                         tc_gemm_tiles(g.m, g.n, ch, 512, false) < sms);
+    const bool maybe_small = !f32 && total <= ch && (tc_gemm_tiles(g.m, g.n, ch, 128, false) < 2LL * sms ||
+                                                     tc_gemm_tiles(g.m, g.n, ch, 512, false) < sms);
     if (maybe_small) small_need = std::max(small_need, align256(L.total));
   }
   *bytes = need + 3 * small_need + align256(4 * sizeof(void*) * static_cast<size_t>(count));

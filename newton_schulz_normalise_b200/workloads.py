@@ -78,6 +78,9 @@ WORKLOADS = {
     # the skewed set's tiny group on its own (the resident small-matrix kernel)
     "batch512-64x256-bf16": Workload(
         "batch512-64x256-bf16", ((64, 256, 512),), seed=3),
+    # the skewed set's medium group on its own (the resident medium-matrix kernel)
+    "batch128-256x1024-bf16": Workload(
+        "batch128-256x1024-bf16", ((256, 1024, 128),), seed=3),
     # Llama-style 8B matrix set: 32 layers of q, k, v, o, gate, up, down
     "llama8b-matrices-bf16": Workload(
         "llama8b-matrices-bf16", _LLAMA8B_LAYER, seed=4, interleave=32),

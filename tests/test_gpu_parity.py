@@ -329,3 +329,50 @@ def test_tall_momentum_vector_path(dmuon_lib, pdt):
         check_momentum(Bn[i], Gs[i], Ms[i], 0.95)
         _, Oo = oracle_update(Gs[i], Ms[i])
         assert rel_fro(to64(Os[i]), Oo) <= tol, (shapes[i], rel_fro(to64(Os[i]), Oo))
+
+
+@pytest.mark.parametrize("pdt,shapes,variant", [
+    ("bf16", [(300, 700)] * 2 + [(700, 300)] * 3, "direct"),
+    ("bf16", [(300, 700)] * 2 + [(700, 300)] * 3, "gram"),
+    ("bf16", [(64, 256)] * 3 + [(256, 64)] * 2, "batched"),
+    ("bf16", [(200, 700), (700, 200)], "batched"),
+    ("f32", [(256, 512), (512, 256)] * 2, "batched"),
+    ("f32", [(96, 200), (200, 96)], "direct"),
+], ids=["direct", "gram", "small", "medium", "f32-resident", "f32-simt"])
+def test_weight_and_transposed_weight_share_one_group(dmuon_lib, monkeypatch, pdt, shapes, variant):
+    """Matrices stored m x n and n x m share every Newton-Schulz product (one
+    launch per product serves both) and differ only in the momentum kernel
+    and the final write.  Against the oracle, and bit for bit against one
+    call per orientation with the same forced form and tile."""
+    monkeypatch.setenv("DMUON_TILE", "512")
+    std = 0.02 if pdt == "f32" else 1e-3
+    Ws, Gs, Ms = make_inputs(shapes, seed=71, pdt=pdt, m_std=std, g_std=std)
+    Os, Bn = gpu_update(dmuon_lib, Gs, Ms, variant=variant)
+    tol = F32_TOL if pdt == "f32" else BF16_TOL
+    for i in range(len(shapes)):
+        _, Oo = oracle_update(Gs[i], Ms[i])
+        assert rel_fro(to64(Os[i]), Oo) <= tol, (shapes[i], rel_fro(to64(Os[i]), Oo))
+        check_momentum(Bn[i], Gs[i], Ms[i], 0.95)
+    wide = [i for i, (r, c) in enumerate(shapes) if r <= c]
+    tall = [i for i, (r, c) in enumerate(shapes) if r > c]
+    for part in (wide, tall):
+        Op, Bp = gpu_update(dmuon_lib, [Gs[i] for i in part], [Ms[i] for i in part], variant=variant)
+        for j, i in enumerate(part):
+            assert torch.equal(Op[j], Os[i]), (shapes[i], variant)
+            assert torch.equal(Bp[j], Bn[i])
+    # the fused write of the step on the same group
+    Wg, _ = gpu_step(dmuon_lib, Ws, Gs, Ms, variant=variant)
+    for i, (r, c) in enumerate(shapes):
+        w_apply = ora.apply_update(to64(Ws[i]), to64(Os[i]), 0.02, 0.1)
+        terms = np.abs(0.998 * to64(Ws[i])) + np.abs(0.02 * ora.rms_scale(r, c) * to64(Os[i]))
+        unit = 2.0 ** -21 if pdt == "f32" else 2.0 ** -8
+        assert np.all(np.abs(to64(Wg[i]) - w_apply) <= np.abs(w_apply) * unit + terms * 2.0 ** -21 + 1e-30), i
+
+
+def test_mixed_orientation_zero_steps(dmuon_lib):
+    shapes = [(48, 80), (80, 48), (48, 80)]
+    Ws, Gs, Ms = make_inputs(shapes, seed=72, m_std=1e-3)
+    Os, _ = gpu_update(dmuon_lib, Gs, Ms, steps=0)
+    for i in range(len(shapes)):
+        _, Oo = oracle_update(Gs[i], Ms[i], steps=0)
+        assert rel_fro(to64(Os[i]), Oo) <= BF16_TOL, i
