@@ -8,6 +8,10 @@
 // memory: the fp32 workloads are single matrices of a few hundred rows, so
 // small tiles are what spreads a product over the SMs; when even those leave
 // SMs idle, K is split over a cluster of 2-8 CTAs (simt_gemm_splitk_kernel).
+// Consecutive products are launched with programmatic dependent launch: each
+// kernel lets the next one launch as soon as all its own CTAs are running,
+// and waits for the previous one's results before reading anything, so a
+// launch's start-up overlaps the previous product's tail.
 #include "internal.h"
 
 namespace dmuon {
@@ -21,6 +25,8 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const float* __restrict_
                                                         int b_kmajor, int M, int N, int K, const Epilogue epi) {
   __shared__ float As[TK][TM + 1];
   __shared__ float Bs[TK][TN + 1];
+  grid_dep_wait();    // the previous product's results are complete and visible
+  grid_dep_launch();  // the next product may start launching
   const int l = blockIdx.z;
   const int m0 = blockIdx.y * TM, n0 = blockIdx.x * TN;
   const int tid = threadIdx.x;
@@ -89,6 +95,8 @@ __global__ void __launch_bounds__(256) simt_gemm_splitk_kernel(const float* __re
   __shared__ float As[TK][TM + 1];
   __shared__ float Bs[TK][TN + 1];
   __shared__ float part[TM][TN];
+  grid_dep_wait();
+  grid_dep_launch();
   const int l = blockIdx.z;
   const int r = static_cast<int>(cluster_rank());  // K slice of this CTA
   const int m0 = blockIdx.y * TM, n0 = (blockIdx.x / S) * TN;
@@ -171,20 +179,29 @@ cudaError_t launch_simt_gemm(const SimtGemm& g, cudaStream_t s) {
     cfg.gridDim = dim3(static_cast<unsigned>(tiles_n * S), static_cast<unsigned>(tiles_m), static_cast<unsigned>(g.batch));
     cfg.blockDim = dim3(256);
     cfg.stream = s;
-    cudaLaunchAttribute attr;
-    attr.id = cudaLaunchAttributeClusterDimension;
-    attr.val.clusterDim.x = static_cast<unsigned>(S);
-    attr.val.clusterDim.y = 1;
-    attr.val.clusterDim.z = 1;
-    cfg.attrs = &attr;
-    cfg.numAttrs = 1;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, simt_gemm_splitk_kernel, g.A, g.lda, g.sa, g.B, g.ldb, g.sb, g.b_kmajor ? 1 : 0,
                               g.M, g.N, g.K, S, ks, g.epi);
   }
-  dim3 grid(tiles_n, tiles_m, g.batch);
-  simt_gemm_kernel<<<grid, 256, 0, s>>>(g.A, g.lda, g.sa, g.B, g.ldb, g.sb, g.b_kmajor ? 1 : 0, g.M, g.N, g.K,
-                                        g.epi);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles_n), static_cast<unsigned>(tiles_m), static_cast<unsigned>(g.batch));
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr.val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, simt_gemm_kernel, g.A, g.lda, g.sa, g.B, g.ldb, g.sb, g.b_kmajor ? 1 : 0, g.M, g.N,
+                            g.K, g.epi);
 }
 
 }  // namespace dmuon

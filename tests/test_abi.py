@@ -77,6 +77,11 @@ def test_host_validation_rejects_before_any_launch(dmuon_lib):
     o = L.options()
     o.variant = 9
     assert _call_step(L, opts=o) == L.DMUON_ERR_INVALID
+    # the size limits: a side above 2^20, or more than 2^31 elements in one matrix
+    assert _call_step(L, shapes=((1 << 20) + 1, 8)) == L.DMUON_ERR_INVALID
+    assert _call_step(L, shapes=(8, (1 << 20) + 1)) == L.DMUON_ERR_INVALID
+    assert _call_step(L, shapes=(1 << 16, (1 << 15) + 1)) == L.DMUON_ERR_INVALID
+    assert "too large" in L.last_error()
 
 
 def test_workspace_size_is_host_only_and_monotone(dmuon_lib):

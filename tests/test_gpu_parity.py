@@ -376,3 +376,18 @@ def test_mixed_orientation_zero_steps(dmuon_lib):
     for i in range(len(shapes)):
         _, Oo = oracle_update(Gs[i], Ms[i], steps=0)
         assert rel_fro(to64(Os[i]), Oo) <= BF16_TOL, i
+
+
+@pytest.mark.parametrize("pdt", ["bf16", "f32"])
+def test_degenerate_shapes(dmuon_lib, pdt):
+    """A 1 x 1 weight (the iteration acts on one singular value), 1 x 2 and
+    2 x 1, a 3 x 3, and a single row far wider than any tile."""
+    shapes = [(1, 1), (1, 2), (2, 1), (3, 3), (1, 20000)]
+    std = 0.02 if pdt == "f32" else 1e-3
+    Ws, Gs, Ms = make_inputs(shapes, seed=75, pdt=pdt, m_std=std, g_std=std)
+    Os, Bn = gpu_update(dmuon_lib, Gs, Ms)
+    tol = F32_TOL if pdt == "f32" else BF16_TOL
+    for i in range(len(shapes)):
+        _, Oo = oracle_update(Gs[i], Ms[i])
+        assert rel_fro(to64(Os[i]), Oo) <= tol, (shapes[i], rel_fro(to64(Os[i]), Oo))
+        check_momentum(Bn[i], Gs[i], Ms[i], 0.95)
