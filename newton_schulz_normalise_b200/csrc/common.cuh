@@ -260,10 +260,10 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
-// Instruction descriptor: kind::f16, bf16 A and B, fp32 D, A K-major,
-// B K-major or MN-major, shape M x N.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+// Instruction descriptor: kind::f16, bf16 A and B, fp32 D, A K-major or
+// MN-major, B K-major or MN-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major, bool a_mn_major = false) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
@@ -296,6 +296,7 @@ struct Epilogue {
   int sym;                       // EPI_STORE of a symmetric M x M result: only the blocks on
                                  // and above the block diagonal run; blocks above it are
                                  // also stored mirrored (see the tensor-core kernels)
+                                 // unless the launch keeps the result upper-only
 };
 
 __device__ __forceinline__ float load_elem(const void* p, long long i, int is_f32) {

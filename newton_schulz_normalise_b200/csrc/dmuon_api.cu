@@ -403,15 +403,17 @@ T* at(const Chunk& ch, size_t off) {
 // sym: the M x M result is symmetric; the tensor-core kernels compute only the
 // tiles that meet the upper triangle and mirror them (FLOPs counted for the
 // computed tiles only).
+// upper (CTA-pair tiles only, see TcGemm): which symmetric operands and
+// result are kept as their blocks on and above the diagonal.
 int gemm(DeviceCtx& c, int cnt, bool f32, int tile, bool sym, const void* A, long long lda, long long sa,
          const void* B, long long ldb, long long sb, bool b_kmajor, int M, int N, int K, const Epilogue& e,
-         cudaStream_t s) {
+         cudaStream_t s, int upper = 0) {
   cudaError_t err;
   if (!f32) {
     const long long tiles = tc_gemm_tiles(M, N, cnt, tile, sym);
     const long long dense = tc_gemm_tiles(M, N, cnt, tile, false);
     const double flops = 2.0 * M * N * static_cast<double>(K) * cnt * static_cast<double>(tiles) / dense;
-    TcGemm t{A, lda, sa, B, ldb, sb, b_kmajor, M, N, K, cnt, tile, sym, e};
+    TcGemm t{A, lda, sa, B, ldb, sb, b_kmajor, M, N, K, cnt, tile, sym, e, tile == 512 ? upper : 0};
     err = launch_k(KIND_TC_GEMM, flops, 0.0, s, [&] { return launch_tc_gemm(t, s, c.err_dev, c.num_sms); });
   } else {
     const double flops = 2.0 * M * N * static_cast<double>(K) * cnt;
@@ -567,6 +569,12 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
       return DMUON_OK;
     });
   }
+  // On CTA-pair tiles every symmetric m x m matrix of the chain is kept as its
+  // 256 x 256 blocks on and above the diagonal (no mirrored copy): the
+  // products that make one pass UP_OUT, and every product that reads one as
+  // its left (UP_A) or right (UP_B) operand reads the blocks below the
+  // diagonal from the stored blocks across it.
+  constexpr int UP_A = 1, UP_B = 2, UP_OUT = 4;
   // The last product O = scale * Aop Bx (m x n, K = m, Bx the MN-major iterate),
   // once per orientation part with its epilogue.
   auto final_product = [&](const void* Aop, const void* Bx, bool scale) -> int {
@@ -578,7 +586,7 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
       fin.C = nullptr;
       return gemm(c, nn, f32, tile, false, static_cast<const uint8_t*>(Aop) + static_cast<size_t>(off) * sq * g.esz,
                   g.ldm, sq, static_cast<const uint8_t*>(Bx) + static_cast<size_t>(off) * sx * g.esz, g.ldx, sx, false,
-                  m, n, m, fin, s);
+                  m, n, m, fin, s, UP_A);
     });
   };
   if (variant == DMUON_VARIANT_GRAM) {
@@ -592,7 +600,8 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
     void* T = at<void>(ch, ch.L.T);
     void* Q[2] = {at<void>(ch, ch.L.Q0), at<void>(ch, ch.L.Q1)};
     // G = s^2 U U^T  (A_0): both operands are rows of U (K-major)
-    rc = gemm(c, cnt, f32, tile, true, X0, g.ldx, sx, X0, g.ldx, sx, true, m, m, n, store_epi(A, g.ldm, sq, f32, 1.f, s2v), s);
+    rc = gemm(c, cnt, f32, tile, true, X0, g.ldx, sx, X0, g.ldx, sx, true, m, m, n, store_epi(A, g.ldm, sq, f32, 1.f, s2v), s,
+              UP_OUT);
     if (rc) return rc;
     int qi = 0;
     for (int k = 0; k < h.steps; ++k) {
@@ -604,20 +613,20 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
       ep.sc = sq;
       ep.beta = h.b;
       ep.diag = h.a;
-      rc = gemm(c, cnt, f32, tile, true, A, g.ldm, sq, A, g.ldm, sq, false, m, m, m, ep, s);
+      rc = gemm(c, cnt, f32, tile, true, A, g.ldm, sq, A, g.ldm, sq, false, m, m, m, ep, s, UP_A | UP_B | UP_OUT);
       if (rc) return rc;
       if (k > 0) {  // Q_{k+1} = P_k Q_k
         rc = gemm(c, cnt, f32, tile, true, Pk, g.ldm, sq, Q[qi], g.ldm, sq, false, m, m, m,
-                  store_epi(Q[qi ^ 1], g.ldm, sq, f32, 1.f, nullptr), s);
+                  store_epi(Q[qi ^ 1], g.ldm, sq, f32, 1.f, nullptr), s, UP_A | UP_B | UP_OUT);
         if (rc) return rc;
         qi ^= 1;
       }
       if (k < h.steps - 1) {  // A_{k+1} = P_k A_k P_k
         rc = gemm(c, cnt, f32, tile, true, Pk, g.ldm, sq, A, g.ldm, sq, false, m, m, m,
-                  store_epi(T, g.ldm, sq, f32, 1.f, nullptr), s);
+                  store_epi(T, g.ldm, sq, f32, 1.f, nullptr), s, UP_A | UP_B | UP_OUT);
         if (rc) return rc;
         rc = gemm(c, cnt, f32, tile, true, T, g.ldm, sq, Pk, g.ldm, sq, false, m, m, m,
-                  store_epi(A, g.ldm, sq, f32, 1.f, nullptr), s);
+                  store_epi(A, g.ldm, sq, f32, 1.f, nullptr), s, UP_A | UP_B | UP_OUT);
         if (rc) return rc;
       }
     }
@@ -638,7 +647,7 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
     const bool last = (k == h.steps - 1);
     // A = X X^T  (s^2 folded in on the first step)
     rc = gemm(c, cnt, f32, tile, true, cur, g.ldx, sx, cur, g.ldx, sx, true, m, m, n,
-              store_epi(A, g.ldm, sq, f32, 1.f, first ? s2v : nullptr), s);
+              store_epi(A, g.ldm, sq, f32, 1.f, first ? s2v : nullptr), s, UP_OUT);
     if (rc) return rc;
     // P = c A A + b A + a I   (right operand as stored, see the Gram form)
     Epilogue ep = store_epi(P, g.ldm, sq, f32, h.c, nullptr);
@@ -647,13 +656,13 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
     ep.sc = sq;
     ep.beta = h.b;
     ep.diag = h.a;
-    rc = gemm(c, cnt, f32, tile, true, A, g.ldm, sq, A, g.ldm, sq, false, m, m, m, ep, s);
+    rc = gemm(c, cnt, f32, tile, true, A, g.ldm, sq, A, g.ldm, sq, false, m, m, m, ep, s, UP_A | UP_B | UP_OUT);
     if (rc) return rc;
     // X' = P X   (times s on the first step)
     if (last) return final_product(P, cur, first);
     void* nxt = bufs[k & 1];
     rc = gemm(c, cnt, f32, tile, false, P, g.ldm, sq, cur, g.ldx, sx, false, m, n, m,
-              store_epi(nxt, g.ldx, sx, f32, 1.f, first ? sv : nullptr), s);
+              store_epi(nxt, g.ldx, sx, f32, 1.f, first ? sv : nullptr), s, UP_A);
     if (rc) return rc;
     cur = nxt;
   }

@@ -496,12 +496,27 @@ constexpr int P_STAGES = 5;
 constexpr int P_TMEM_COLS = 2 * P_BN;  // two 256-column accumulators = all 512 columns
 constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + STG_TOTAL + 1024 + 256;
 
+// Symmetric operands stored upper-only (flags).  A chain of products on
+// pair tiles keeps each symmetric result as its 256 x 256 blocks on and above
+// the block diagonal, without the mirrored copy.  A consumer reads a sub-tile
+// that lies below the diagonal from the stored block across it, transposed:
+//   A operand (rows of block tm, a 64-deep k block in block kb/4 < tm):
+//     stored rows k, columns m -> two 64 x 64 boxes, the MN-major A layout;
+//   B operand taken as stored, MN-major (k block in block kb/4 > tn):
+//     stored rows n, columns k -> one 64 x 128 box, the K-major B layout.
+// The MMA of that k block takes the matching descriptors and major-ness; the
+// values are the ones the mirror would have held, so results are unchanged.
+constexpr int SYM_A = 1;    // A operand is a symmetric matrix stored upper-only
+constexpr int SYM_B = 2;    // B operand (as stored) is one
+constexpr int SYM_OUT = 4;  // the symmetric result is stored upper-only (no mirror)
+
 template <bool B_MN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc_gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
-                    const __grid_constant__ CUtensorMap tmDm, const Epilogue epi, int M, int N, int K, int batch,
-                    int sym, long long per_mat, int staged, int* err) {
+                    const __grid_constant__ CUtensorMap tmDm, const __grid_constant__ CUtensorMap tmAt,
+                    const __grid_constant__ CUtensorMap tmBt, const Epilogue epi, int M, int N, int K, int batch,
+                    int sym, long long per_mat, int staged, int flags, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stg = smem + P_STAGES * P_STAGE_BYTES;
@@ -533,6 +548,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (flags & SYM_A) tma_prefetch_desc(&tmAt);
+    if ((flags & SYM_B) && B_MN) tma_prefetch_desc(&tmBt);
   }
   if (warp == 2) {
     tmem_alloc2(tmem_slot, P_TMEM_COLS);
@@ -567,9 +584,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         uint8_t* sb = sa + P_A_BYTES;
         const uint32_t fbar = mapa_shared(smem_u32(&full[stage]), 0);
         if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * P_STAGE_BYTES);
-        tma_load_3d_pair(sa, &tmA, fbar, kb * BK, tm * P_BM + static_cast<int>(rank) * BM, l);
+        const int kblk = (kb * BK) / P_BM;  // the 256-block of this k range
+        const int m0 = tm * P_BM + static_cast<int>(rank) * BM;
+        if ((flags & SYM_A) && kblk < tm) {  // below the diagonal: the stored block across it, transposed
+#pragma unroll
+          for (int j = 0; j < BM / 64; ++j)
+            tma_load_3d_pair(sa + j * (BK * 128), &tmAt, fbar, m0 + j * 64, kb * BK, l);
+        } else {
+          tma_load_3d_pair(sa, &tmA, fbar, kb * BK, m0, l);
+        }
         const int n0 = tn * P_BN + static_cast<int>(rank) * (P_BN / 2);
-        if (B_MN) {
+        if (B_MN && (flags & SYM_B) && kblk > tn) {
+          tma_load_3d_pair(sb, &tmBt, fbar, kb * BK, n0, l);
+        } else if (B_MN) {
 #pragma unroll
           for (int j = 0; j < P_BN / 2 / 64; ++j)
             tma_load_3d_pair(sb + j * (BK * 128), &tmB, fbar, n0 + j * 64, kb * BK, l);
@@ -591,12 +618,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
   } else if (warp == 1 && lane == 0 && rank == 0) {
     // ------------------------------------------------ MMA issuer (leader)
-    constexpr uint32_t IDESC = idesc_bf16_f32(P_BM, P_BN, B_MN);
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (long long t = pair; t < total && !*abort; t += npairs) {
+      int l, tm = 0, tn = 0;
+      bool mir;
+      if (flags & (SYM_A | SYM_B)) decode_tile(t, per_mat, tiles_m, tiles_n, P_BM, P_BN, sy, l, tm, tn, mir);
       if (!mbar_wait(&tempty[acc], acc_phase ^ 1, abort)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + acc * P_BN;
@@ -609,12 +638,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         tc_fence_after();
         const uint32_t sa = smem_u32(smem + stage * P_STAGE_BYTES);
         const uint32_t sb = sa + P_A_BYTES;
+        const int kblk = (kb * BK) / P_BM;
+        const bool a_mn = (flags & SYM_A) && kblk < tm;           // A loaded transposed (MN-major)
+        const bool b_mn = B_MN && !((flags & SYM_B) && kblk > tn);  // B as stored (MN-major) or transposed
+        const uint32_t idesc = idesc_bf16_f32(P_BM, P_BN, b_mn, a_mn);
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t adesc = smem_desc_sw128(sa + kk * 32, 16, 1024);
+          const uint64_t adesc =
+              a_mn ? smem_desc_sw128(sa + kk * 16 * 128, BK * 128, 1024) : smem_desc_sw128(sa + kk * 32, 16, 1024);
           const uint64_t bdesc =
-              B_MN ? smem_desc_sw128(sb + kk * 16 * 128, BK * 128, 1024) : smem_desc_sw128(sb + kk * 32, 16, 1024);
-          umma_bf16_pair(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+              b_mn ? smem_desc_sw128(sb + kk * 16 * 128, BK * 128, 1024) : smem_desc_sw128(sb + kk * 32, 16, 1024);
+          umma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
         }
         umma_commit_pair(&empty[stage], 0x3);
         if (++stage == P_STAGES) {
@@ -643,6 +677,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
       int l, tm, tn;
       bool mir;
       decode_tile(t, per_mat, tiles_m, tiles_n, P_BM, P_BN, sy, l, tm, tn, mir);
+      if (flags & SYM_OUT) mir = false;
       const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, abort));
       if (!ok) break;
       tc_fence_after();
@@ -799,6 +834,16 @@ cudaError_t launch_pair(const TcGemm& g, cudaStream_t s, int* dev_err, int num_s
   if (!ok) return cudaErrorInvalidValue;
   CUtensorMap mc = ma, md = ma, mm = ma;
   const int staged = make_stage_maps(g, &mc, &md, &mm) ? 1 : 0;
+  // transposed views of upper-only symmetric operands: A's stored rows k,
+  // columns m in 64 x 64 boxes; B's stored rows n, columns k in 64 x 128 boxes
+  int flags = g.upper & (SYM_A | SYM_B | SYM_OUT);
+  if ((flags & SYM_A) && g.M != g.K) return cudaErrorInvalidValue;
+  if ((flags & SYM_B) && (!B_MN || g.K != g.N)) return cudaErrorInvalidValue;
+  if ((flags & SYM_OUT) && !(g.sym && staged)) flags &= ~SYM_OUT;  // the mirror is written unless staged
+  CUtensorMap mat = ma, mbt = mb;
+  if ((flags & SYM_A) && !make_map(&mat, g.A, g.K, g.M, g.batch, g.lda, g.sa, 64, 64)) return cudaErrorInvalidValue;
+  if ((flags & SYM_B) && !make_map(&mbt, g.B, g.N, g.K, g.batch, g.ldb, g.sb, BK, P_BN / 2))
+    return cudaErrorInvalidValue;
   const long long per_mat = tiles_per_matrix(g.M, g.N, P_BM, P_BN, g.sym);
   const long long tiles = per_mat * g.batch;
   const long long pairs = tiles < max_clusters ? tiles : max_clusters;
@@ -812,8 +857,8 @@ cudaError_t launch_pair(const TcGemm& g, cudaStream_t s, int* dev_err, int num_s
   attr.val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = &attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, tc_gemm2_kernel<B_MN>, ma, mb, mc, md, mm, g.epi, g.M, g.N, g.K, g.batch,
-                            g.sym ? 1 : 0, per_mat, staged, dev_err);
+  return cudaLaunchKernelEx(&cfg, tc_gemm2_kernel<B_MN>, ma, mb, mc, md, mm, mat, mbt, g.epi, g.M, g.N, g.K, g.batch,
+                            g.sym ? 1 : 0, per_mat, staged, flags, dev_err);
 }
 
 }  // namespace

@@ -21,6 +21,11 @@ struct TcGemm {
   int tile;  // 128 / 256: one CTA, 128 x tile output tile; 512: CTA pair, 256 x 256
   bool sym;  // M == N and the result is symmetric: upper-triangle tiles only, mirrored
   Epilogue epi;
+  // CTA pair only (tile 512): symmetric matrices kept as their 256 x 256 blocks
+  // on and above the diagonal.  1: A (M x K, M == K) is one; 2: B as stored
+  // (K x N, K == N, MN-major) is one; 4: the symmetric result is stored that
+  // way (no mirrored copy).  Ignored for other tiles.
+  int upper = 0;
 };
 
 // Same contract in fp32 on the CUDA cores (fp32 path; any leading dims).
