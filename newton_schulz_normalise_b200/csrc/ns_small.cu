@@ -96,6 +96,31 @@ __host__ __device__ constexpr int small_tmem_cols(int n) { return n <= 128 ? 128
 
 constexpr int SM_THREADS = 256;  // 8 warps: two per TMEM lane quarter
 
+// Drains columns [0, limit) of this warp's TMEM lanes in the 32-column chunks
+// half*32, half*32 + 64, ... (the other warp of the lane quarter takes the
+// rest); fn(c0, v) gets each chunk as fp32.  With PAIR two loads are in
+// flight per wait (for passes whose fn needs few registers).
+template <bool PAIR, typename F>
+__device__ __forceinline__ void drain(uint32_t trow, int half, int limit, F&& fn) {
+#pragma unroll 1
+  for (int c0 = half * 32; c0 < limit; c0 += PAIR ? 128 : 64) {
+    uint32_t r0[32], r1[32];
+    const bool two = PAIR && c0 + 64 < limit;  // warp-uniform
+    tmem_ld_32cols_async(trow + c0, r0);
+    if (two) tmem_ld_32cols_async(trow + c0 + 64, r1);
+    tmem_wait_ld();
+    float v[32];
+#pragma unroll
+    for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(r0[t]);
+    fn(c0, v);
+    if (two) {
+#pragma unroll
+      for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(r1[t]);
+      fn(c0 + 64, v);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(SM_THREADS, 2) ns_small_kernel(const SmallArgs p, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -106,6 +131,7 @@ __global__ void __launch_bounds__(SM_THREADS, 2) ns_small_kernel(const SmallArgs
   uint64_t* bar = reinterpret_cast<uint64_t*>(As + 2 * ATOM);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* live = const_cast<int*>(abort) + 1;  // [8]
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int r = tid & (SM_ROWS - 1);    // TMEM lane = tile row of this thread
@@ -123,26 +149,49 @@ __global__ void __launch_bounds__(SM_THREADS, 2) ns_small_kernel(const SmallArgs
     tmem_alloc(tmem_slot, small_tmem_cols(p.n));
     tmem_relinquish();
   }
-  // X0 -> shared (zero rows outside the matrices).  A matrix whose scale s
-  // is not a positive finite number (a NaN or Inf in its gradient) is loaded
-  // as zeros: the stacked products multiply across matrices (0 * NaN = NaN),
-  // so its values must not reach the shared tile; its output is NaN instead.
+  // Which of this block's matrices have a positive finite scale s.  A matrix
+  // whose s is not (a NaN or Inf in its gradient) is loaded as zeros: the
+  // stacked products multiply across matrices (0 * NaN = NaN), so its values
+  // must not reach the shared tile; its output is NaN instead.
+  if (tid < p.g) {
+    const int ll = blockIdx.x * p.g + tid;
+    live[tid] = ll < p.cnt && finite_scale(p.s[ll]);
+  }
+  // The fused update reads every weight of the block at the end: start
+  // bringing them into L2 now, behind the Newton-Schulz steps.
+  if (p.fin.mode == EPI_APPLY) {
+    const int esz = p.fin.w_f32 ? 4 : 2;
+    const long long srows = p.fin.transposed ? p.n : p.m, scols = p.fin.transposed ? p.m : p.n;
+    const long long bytes = ((srows - 1) * p.fin.ldw + scols) * esz;
+    for (int jj = 0; jj < p.g && blockIdx.x * p.g + jj < p.cnt; ++jj) {
+      const uint8_t* w = static_cast<const uint8_t*>(p.fin.W[blockIdx.x * p.g + jj]);
+      for (long long off = static_cast<long long>(tid) * 128; off < bytes; off += SM_THREADS * 128) prefetch_l2(w + off);
+      if (tid == 0) prefetch_l2(w + bytes - 1);
+    }
+  }
+  __syncthreads();
+  // X0 -> shared (zero rows outside the matrices), as 16-byte asynchronous
+  // copies so that all of a thread's loads are in flight at once.
   const int chunks = xatoms * 8;  // 16-byte chunks per row (n padded to 64)
   for (int idx = tid; idx < SM_ROWS * chunks; idx += SM_THREADS) {
     const int rr = idx / chunks, q = idx % chunks;
     const int jj = rr / p.mr, ii = rr % p.mr, ll = blockIdx.x * p.g + jj;
-    uint4 u = make_uint4(0, 0, 0, 0);
-    if (ll < p.cnt && ii < p.m && q * 8 < p.n && finite_scale(p.s[ll])) {
+    uint8_t* dst = Xs + sw128_off(rr, q * 8);
+    if (live[jj] && ii < p.m && q * 8 < p.n) {
       const __nv_bfloat16* src = p.X0 + static_cast<long long>(ll) * p.m * p.ldx + static_cast<long long>(ii) * p.ldx + q * 8;
       if (q * 8 + 8 <= p.n) {
-        u = *reinterpret_cast<const uint4*>(src);
+        cp_async16(smem_u32(dst), src, 16);
       } else {
+        uint4 u = make_uint4(0, 0, 0, 0);
         __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(&u);
         for (int t = 0; t < 8 && q * 8 + t < p.n; ++t) h[t] = src[t];
+        *reinterpret_cast<uint4*>(dst) = u;
       }
+    } else {
+      cp_async16(smem_u32(dst), p.X0, 0);  // zero fill
     }
-    *reinterpret_cast<uint4*>(Xs + sw128_off(rr, q * 8)) = u;
   }
+  cp_async_wait_all();
   fence_proxy_async();
   tc_fence_before();
   __syncthreads();
@@ -167,17 +216,14 @@ __global__ void __launch_bounds__(SM_THREADS, 2) ns_small_kernel(const SmallArgs
     phase ^= 1;
     if (!__syncthreads_and(ok)) break;
     tc_fence_after();
-#pragma unroll 1
-    for (int c0 = half * 32; c0 < SM_ROWS; c0 += 64) {
-      float v[32];
-      tmem_ld_32cols(trow + c0, v);
+    drain<true>(trow, half, SM_ROWS, [&](int c0, float (&v)[32]) {
 #pragma unroll
       for (int t = 0; t < 32; ++t) {
         const bool same = ((c0 + t) / p.mr) == j;
         v[t] = same ? (first ? s2l * v[t] : v[t]) : 0.f;  // block-diagonal A
       }
       put_row32(As, r, c0, v);
-    }
+    });
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
@@ -188,15 +234,13 @@ __global__ void __launch_bounds__(SM_THREADS, 2) ns_small_kernel(const SmallArgs
     phase ^= 1;
     if (!__syncthreads_and(ok)) break;
     tc_fence_after();
-#pragma unroll 1
-    for (int c0 = half * 32; c0 < SM_ROWS; c0 += 64) {
-      float v[32], av[32];
-      tmem_ld_32cols(trow + c0, v);
+    drain<false>(trow, half, SM_ROWS, [&](int c0, float (&v)[32]) {
+      float av[32];
       get_row32(As, r, c0, av);  // this row of A, then the same row of P over it
 #pragma unroll
       for (int t = 0; t < 32; ++t) v[t] = p.c * v[t] + p.b * av[t] + ((c0 + t) == r ? p.a : 0.f);
       put_row32(Ps, r, c0, v);
-    }
+    });
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
@@ -224,22 +268,20 @@ __global__ void __launch_bounds__(SM_THREADS, 2) ns_small_kernel(const SmallArgs
     if (!__syncthreads_and(ok)) break;
     tc_fence_after();
     const float alpha = first ? sl : 1.f;
-#pragma unroll 1
-    for (int c0 = half * 32; c0 < npad; c0 += 64) {
-      float v[32];
-      tmem_ld_32cols(trow + c0, v);
+    if (!last) {
+      drain<false>(trow, half, npad, [&](int c0, float (&v)[32]) {
 #pragma unroll
-      for (int t = 0; t < 32; ++t) v[t] *= alpha;
-      if (!last) {
+        for (int t = 0; t < 32; ++t) v[t] *= alpha;
         put_row32(Xs, r, c0, v);
-      } else if (valid_row && c0 < p.n) {
-        // fin: alpha 1 (the step's scale is applied above), per-matrix pointers
-        if (poisoned) {
+      });
+    } else {
+      drain<false>(trow, half, npad, [&](int c0, float (&v)[32]) {
+        if (!valid_row || c0 >= p.n) return;
+        // fin: alpha 1 (the step's scale is applied here), per-matrix pointers
 #pragma unroll
-          for (int t = 0; t < 32; ++t) v[t] = __int_as_float(0x7fc00000);
-        }
+        for (int t = 0; t < 32; ++t) v[t] = poisoned ? __int_as_float(0x7fc00000) : v[t] * alpha;
         epilogue_row<32>(p.fin, l, i, c0, v, p.m, p.n);
-      }
+      });
     }
     fence_proxy_async();
     tc_fence_before();
