@@ -74,8 +74,9 @@ typedef enum dmuon_variant {
   DMUON_VARIANT_GRAM = 2,    /* iterate on Q (m x m), one m x m x n product at the end */
   DMUON_VARIANT_BATCHED = 3  /* resident, every step in one launch.  bf16, m <= 128, n <= 512: up
                                 to 8 small matrices per CTA, iterate, A and P in shared memory for
-                                all steps.  bf16, other m <= 256, n <= 1024: one CTA pair per
-                                matrix, A and P in shared memory, X streamed over k.  fp32,
+                                all steps.  bf16, other m <= 256, n <= 1024 with 4n >= 5m: one CTA
+                                pair per matrix, the Gram-space chain (A, P, Q, m x m) in shared
+                                memory, X read twice.  fp32,
                                 m <= 1024: one cooperative launch over all SMs, a grid barrier
                                 between products.  Other shapes run as AUTO */
 } dmuon_variant;
@@ -176,8 +177,8 @@ int dmuon_compute_update(const void* const* grads, void* const* momenta,
  * device, with that device current); make that first call before any stream
  * capture.  The address is kept for the life of the process, so
  * cudaDeviceReset while the library is loaded is not supported.
- * Plan: opts->variant == DMUON_VARIANT_BATCHED runs the resident kernel when
- * the shape fits it (bf16, m <= 128, n <= 512); otherwise the call uses the
+ * Plan: opts->variant == DMUON_VARIANT_BATCHED runs a resident kernel when
+ * the shape fits one (see DMUON_VARIANT_BATCHED); otherwise the call uses the
  * plan the autotuner cached for this shape (count 1) when there is one, else
  * the direct form; it never autotunes.
  * All calls share the one array and it keeps the last call's contents (each

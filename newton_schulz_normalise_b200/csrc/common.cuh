@@ -414,41 +414,64 @@ __device__ __forceinline__ void epilogue_row(const Epilogue& e, int l, int row, 
     void* W = e.W[l];
     if (!e.transposed) {
       const long long wbase = static_cast<long long>(row) * e.ldw + col;
+      // every load is issued before the first store, so the row's loads are
+      // in flight together (a store may alias a later load for the compiler)
       if (!e.w_f32 && full && (CNT % 8 == 0) && ((wbase & 7) == 0) &&
           ((reinterpret_cast<uintptr_t>(W) & 15) == 0)) {
         uint4* wp = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(W) + wbase);
+        uint4 u[CNT / 8 > 0 ? CNT / 8 : 1];
+#pragma unroll
+        for (int q = 0; q < CNT / 8; ++q) u[q] = wp[q];
 #pragma unroll
         for (int q = 0; q < CNT / 8; ++q) {
-          uint4 u = wp[q];
-          __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+          __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u[q]);
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
             float2 w = __bfloat1622float2(h[t]);
             h[t] = __floats2bfloat162_rn(e.decay * w.x - e.lr_scale * o[q * 8 + 2 * t],
                                          e.decay * w.y - e.lr_scale * o[q * 8 + 2 * t + 1]);
           }
-          wp[q] = u;
+          wp[q] = u[q];
         }
       } else {
+        constexpr int G = CNT < 16 ? CNT : 16;  // loads in flight per group (register budget)
 #pragma unroll
-        for (int j = 0; j < CNT; ++j)
-          if (col + j < N) {
-            const long long i = wbase + j;
-            store_elem(W, i, e.decay * load_elem(W, i, e.w_f32) - e.lr_scale * o[j], e.w_f32);
-          }
+        for (int j0 = 0; j0 < CNT; j0 += G) {
+          float w[G];
+#pragma unroll
+          for (int j = 0; j < G; ++j) w[j] = (col + j0 + j < N) ? load_elem(W, wbase + j0 + j, e.w_f32) : 0.f;
+#pragma unroll
+          for (int j = 0; j < G; ++j)
+            if (col + j0 + j < N) store_elem(W, wbase + j0 + j, e.decay * w[j] - e.lr_scale * o[j0 + j], e.w_f32);
+        }
       }
     } else {
       // iterate element (row, col+j) is stored element (col+j, row): lanes of
       // a warp hold consecutive rows, so each j is a coalesced row segment.
+      constexpr int G = CNT < 16 ? CNT : 16;
 #pragma unroll
-      for (int j = 0; j < CNT; ++j)
-        if (col + j < N) {
-          const long long i = static_cast<long long>(col + j) * e.ldw + row;
-          store_elem(W, i, e.decay * load_elem(W, i, e.w_f32) - e.lr_scale * o[j], e.w_f32);
-        }
+      for (int j0 = 0; j0 < CNT; j0 += G) {
+        float w[G];
+#pragma unroll
+        for (int j = 0; j < G; ++j)
+          w[j] = (col + j0 + j < N) ? load_elem(W, static_cast<long long>(col + j0 + j) * e.ldw + row, e.w_f32) : 0.f;
+#pragma unroll
+        for (int j = 0; j < G; ++j)
+          if (col + j0 + j < N)
+            store_elem(W, static_cast<long long>(col + j0 + j) * e.ldw + row, e.decay * w[j] - e.lr_scale * o[j0 + j],
+                       e.w_f32);
+      }
     }
   } else {  // EPI_OUT
     float* out = e.Out[l];
+    const long long obase = static_cast<long long>(row) * e.ldw + col;
+    if (!e.transposed && full && (CNT % 4 == 0) && ((obase & 3) == 0) &&
+        ((reinterpret_cast<uintptr_t>(out) & 15) == 0)) {
+#pragma unroll
+      for (int q = 0; q < CNT / 4; ++q)
+        reinterpret_cast<float4*>(out + obase)[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+      return;
+    }
 #pragma unroll
     for (int j = 0; j < CNT; ++j)
       if (col + j < N) {

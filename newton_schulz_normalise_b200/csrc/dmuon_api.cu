@@ -550,8 +550,8 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
   if (variant == DMUON_VARIANT_BATCHED && !ns_small_supported(m, n)) {  // bf16, medium: one CTA pair per matrix
     return parts([&](int off, int nn, Epilogue fin) -> int {
       cudaError_t e = launch_k(KIND_TC_GEMM, ns_mid_flops(m, n, h.steps, nn), 0.0, s, [&] {
-        return launch_ns_mid(xoff(off), at<void>(ch, ch.L.Xp), g.ldx, sv + off, s2v + off, nn, m, n, h.steps, h.a,
-                             h.b, h.c, fin, s, c.err_dev, c.num_sms);
+        return launch_ns_mid(xoff(off), g.ldx, sv + off, s2v + off, nn, m, n, h.steps, h.a, h.b, h.c, fin, s,
+                             c.err_dev, c.num_sms);
       });
       if (e != cudaSuccess) return fail(DMUON_ERR_CUDA, "resident medium-matrix kernel: %s", cudaGetErrorString(e));
       return DMUON_OK;
@@ -1678,7 +1678,9 @@ int dmuon_cache_load(const char* path) {
   int f32, steps, cnt, var, tile;
   double cost;
   while (fscanf(f, "%lld %lld %d %d %d %d %d %lf", &rr, &cc, &f32, &steps, &cnt, &var, &tile, &cost) == 8) {
-    if (rr <= 0 || cc <= 0 || cnt <= 0 || var < 1 || var > 3 || (tile != 128 && tile != 256 && tile != 512)) {
+    if (rr <= 0 || cc <= 0 || cnt <= 0 || var < 1 || var > 3 || (tile != 128 && tile != 256 && tile != 512) ||
+        rr > cc || rr > INT32_MAX || cc > INT32_MAX ||
+        (var == DMUON_VARIANT_BATCHED && !resident_supported(f32 != 0, static_cast<int>(rr), static_cast<int>(cc)))) {
       fclose(f);
       return fail(DMUON_ERR_INVALID, "%s: malformed entry", path);
     }

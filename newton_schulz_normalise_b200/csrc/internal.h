@@ -112,13 +112,12 @@ bool ns_f32_supported(int m, int n);
 cudaError_t launch_ns_f32(const NsF32& g, cudaStream_t st, int* err, int num_sms);
 
 // Resident Newton-Schulz for medium bf16 matrices (128 < m <= 256, or m <= 128
-// with 512 < n; n <= 1024), direct form: one CTA pair per matrix, A and P in
-// shared memory for all steps, X streamed over k from the scratch.  X0 is
-// read, never written; Xw ([cnt][m][ldx], same layout) holds the iterate
-// from the second step on.  Ends with `fin`.
+// with 512 < n; n <= 1024), Gram form: one CTA pair per matrix, the m x m
+// chain (A, P, Q) in shared memory, X0 ([cnt][m][ldx]) read twice, never
+// written.  Ends with `fin`.
 bool ns_mid_supported(int m, int n);
-cudaError_t launch_ns_mid(const void* X0, void* Xw, long long ldx, const float* s, const float* s2, int cnt, int m,
-                          int n, int steps, float a, float b, float c, const Epilogue& fin, cudaStream_t st, int* err,
+cudaError_t launch_ns_mid(const void* X0, long long ldx, const float* s, const float* s2, int cnt, int m, int n,
+                          int steps, float a, float b, float c, const Epilogue& fin, cudaStream_t st, int* err,
                           int num_sms);
 double ns_mid_flops(int m, int n, int steps, int cnt);
 

@@ -272,19 +272,22 @@ def test_fp32_resident_nonfinite_stays_in_its_matrix(dmuon_lib):
 
 
 @pytest.mark.parametrize("shapes", [[(256, 1024)] * 3, [(200, 700)] * 2, [(1024, 256)], [(129, 300)], [(100, 900)],
-                                    [(256, 256)] * 2, [(250, 1000)]],
-                         ids=["256x1024x3", "200x700x2", "1024x256", "129x300", "100x900", "256x256x2", "250x1000"])
+                                    [(200, 256)] * 2, [(250, 1000)]],
+                         ids=["256x1024x3", "200x700x2", "1024x256", "129x300", "100x900", "200x256x2", "250x1000"])
 def test_resident_medium_kernel(dmuon_lib, shapes):
-    """The medium resident kernel (one CTA pair per matrix, A and P on chip,
-    X streamed over k, all steps in one launch) against the oracle and the
-    direct form it restates; then its fused parameter write."""
+    """The medium resident kernel (one CTA pair per matrix, the Gram-space
+    chain on chip, X read twice, all steps in one launch) against the oracle
+    and the Gram form of the batched launches it restates; then its fused
+    parameter write."""
     Ws, Gs, Ms = make_inputs(shapes, seed=97, m_std=1e-3)
     Ob, Bb = gpu_update(dmuon_lib, Gs, Ms, variant="batched")
-    Od, _ = gpu_update(dmuon_lib, Gs, Ms, variant="direct")
+    Og, _ = gpu_update(dmuon_lib, Gs, Ms, variant="gram")
     for i in range(len(shapes)):
         _, Oo = oracle_update(Gs[i], Ms[i])
         assert rel_fro(to64(Ob[i]), Oo) <= BF16_TOL, (i, rel_fro(to64(Ob[i]), Oo))
-        assert rel_fro(to64(Ob[i]), to64(Od[i])) <= 1e-2, i
+        # near n = 1.25 m (200 x 256) both Gram forms sit 1.7e-2 from the
+        # oracle and 1.4e-2 from each other; elsewhere within 0.8e-2
+        assert rel_fro(to64(Ob[i]), to64(Og[i])) <= 2e-2, (i, rel_fro(to64(Ob[i]), to64(Og[i])))
         check_momentum(Bb[i], Gs[i], Ms[i], 0.95)
     Wg, _ = gpu_step(dmuon_lib, Ws, Gs, Ms, variant="batched")
     for i, (r, c) in enumerate(shapes):
