@@ -8,6 +8,8 @@
 // memory: the fp32 workloads are single matrices of a few hundred rows, so
 // small tiles are what spreads a product over the SMs; when even those leave
 // SMs idle, K is split over a cluster of 2-8 CTAs (simt_gemm_splitk_kernel).
+// Each slice's loads go to registers one slice ahead, so they are in flight
+// while the previous slice is multiplied.
 // Consecutive products are launched with programmatic dependent launch: each
 // kernel lets the next one launch as soon as all its own CTAs are running,
 // and waits for the previous one's results before reading anything, so a
@@ -19,6 +21,59 @@ namespace dmuon {
 namespace {
 
 constexpr int TM = 32, TN = 32, TK = 32;
+
+// Loads the A tile (32 rows x 32 k, k contiguous: coalesced along k) and the
+// B tile (32 k x 32 columns) of the slice starting at k0 into registers,
+// zero outside the matrix and at or beyond k_end.
+__device__ __forceinline__ void fetch_tiles(const float* Ab, long long lda, const float* Bb, long long ldb, int b_kmajor,
+                                            int M, int N, int k_end, int m0, int n0, int k0, int tid,
+                                            float (&ra)[TM * TK / 256], float (&rb)[TN * TK / 256]) {
+#pragma unroll
+  for (int u = 0; u < TM * TK / 256; ++u) {
+    const int i = tid + 256 * u;
+    const int r = i / TK, k = i % TK;
+    const int gr = m0 + r, gk = k0 + k;
+    ra[u] = (gr < M && gk < k_end) ? Ab[static_cast<long long>(gr) * lda + gk] : 0.f;
+  }
+#pragma unroll
+  for (int u = 0; u < TN * TK / 256; ++u) {
+    const int i = tid + 256 * u;
+    const int c = b_kmajor ? i / TK : i % TN, k = b_kmajor ? i % TK : i / TN;
+    const int gc = n0 + c, gk = k0 + k;
+    rb[u] = (gc < N && gk < k_end)
+                ? (b_kmajor ? Bb[static_cast<long long>(gc) * ldb + gk] : Bb[static_cast<long long>(gk) * ldb + gc])
+                : 0.f;
+  }
+}
+
+__device__ __forceinline__ void store_tiles(float (&As)[TK][TM + 1], float (&Bs)[TK][TN + 1], int b_kmajor, int tid,
+                                            const float (&ra)[TM * TK / 256], const float (&rb)[TN * TK / 256]) {
+#pragma unroll
+  for (int u = 0; u < TM * TK / 256; ++u) {
+    const int i = tid + 256 * u;
+    As[i % TK][i / TK] = ra[u];
+  }
+#pragma unroll
+  for (int u = 0; u < TN * TK / 256; ++u) {
+    const int i = tid + 256 * u;
+    const int c = b_kmajor ? i / TK : i % TN, k = b_kmajor ? i % TK : i / TN;
+    Bs[k][c] = rb[u];
+  }
+}
+
+// acc += this thread's 2 x 2 outputs over one staged slice.
+__device__ __forceinline__ void mult_slice(const float (&As)[TK][TM + 1], const float (&Bs)[TK][TN + 1], int tx, int ty,
+                                           float (&acc)[2][2]) {
+#pragma unroll 8
+  for (int k = 0; k < TK; ++k) {
+    const float a0 = As[k][ty * 2], a1 = As[k][ty * 2 + 1];
+    const float b0 = Bs[k][tx * 2], b1 = Bs[k][tx * 2 + 1];
+    acc[0][0] = fmaf(a0, b0, acc[0][0]);
+    acc[0][1] = fmaf(a0, b1, acc[0][1]);
+    acc[1][0] = fmaf(a1, b0, acc[1][0]);
+    acc[1][1] = fmaf(a1, b1, acc[1][1]);
+  }
+}
 
 __global__ void __launch_bounds__(256) simt_gemm_kernel(const float* __restrict__ A, long long lda, long long sa,
                                                         const float* __restrict__ B, long long ldb, long long sb,
@@ -34,39 +89,14 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const float* __restrict_
   const float* Ab = A + static_cast<long long>(l) * sa;
   const float* Bb = B + static_cast<long long>(l) * sb;
   float acc[2][2] = {};
+  float ra[TM * TK / 256], rb[TN * TK / 256];
+  fetch_tiles(Ab, lda, Bb, ldb, b_kmajor, M, N, K, m0, n0, 0, tid, ra, rb);
   for (int k0 = 0; k0 < K; k0 += TK) {
-    // A tile: 32 rows x 32 k (k contiguous in memory): coalesced along k
-    for (int i = tid; i < TM * TK; i += 256) {
-      const int r = i / TK, k = i % TK;
-      const int gr = m0 + r, gk = k0 + k;
-      As[k][r] = (gr < M && gk < K) ? Ab[static_cast<long long>(gr) * lda + gk] : 0.f;
-    }
-    // B tile: 32 k x 32 columns
-    for (int i = tid; i < TN * TK; i += 256) {
-      int c, k;
-      if (b_kmajor) {
-        c = i / TK;
-        k = i % TK;
-      } else {
-        k = i / TN;
-        c = i % TN;
-      }
-      const int gc = n0 + c, gk = k0 + k;
-      float v = 0.f;
-      if (gc < N && gk < K)
-        v = b_kmajor ? Bb[static_cast<long long>(gc) * ldb + gk] : Bb[static_cast<long long>(gk) * ldb + gc];
-      Bs[k][c] = v;
-    }
+    store_tiles(As, Bs, b_kmajor, tid, ra, rb);
     __syncthreads();
-#pragma unroll 8
-    for (int k = 0; k < TK; ++k) {
-      const float a0 = As[k][ty * 2], a1 = As[k][ty * 2 + 1];
-      const float b0 = Bs[k][tx * 2], b1 = Bs[k][tx * 2 + 1];
-      acc[0][0] = fmaf(a0, b0, acc[0][0]);
-      acc[0][1] = fmaf(a0, b1, acc[0][1]);
-      acc[1][0] = fmaf(a1, b0, acc[1][0]);
-      acc[1][1] = fmaf(a1, b1, acc[1][1]);
-    }
+    // the next slice's loads are in flight while this one is multiplied
+    if (k0 + TK < K) fetch_tiles(Ab, lda, Bb, ldb, b_kmajor, M, N, K, m0, n0, k0 + TK, tid, ra, rb);
+    mult_slice(As, Bs, tx, ty, acc);
     __syncthreads();
   }
   const int col = n0 + tx * 2;
@@ -106,37 +136,13 @@ __global__ void __launch_bounds__(256) simt_gemm_splitk_kernel(const float* __re
   const float* Bb = B + static_cast<long long>(l) * sb;
   const int k_lo = r * ks, k_hi = min(K, k_lo + ks);
   float acc[2][2] = {};
+  float ra[TM * TK / 256], rb[TN * TK / 256];
+  if (k_lo < k_hi) fetch_tiles(Ab, lda, Bb, ldb, b_kmajor, M, N, k_hi, m0, n0, k_lo, tid, ra, rb);
   for (int k0 = k_lo; k0 < k_hi; k0 += TK) {
-    for (int i = tid; i < TM * TK; i += 256) {
-      const int rr = i / TK, k = i % TK;
-      const int gr = m0 + rr, gk = k0 + k;
-      As[k][rr] = (gr < M && gk < k_hi) ? Ab[static_cast<long long>(gr) * lda + gk] : 0.f;
-    }
-    for (int i = tid; i < TN * TK; i += 256) {
-      int c, k;
-      if (b_kmajor) {
-        c = i / TK;
-        k = i % TK;
-      } else {
-        k = i / TN;
-        c = i % TN;
-      }
-      const int gc = n0 + c, gk = k0 + k;
-      float v = 0.f;
-      if (gc < N && gk < k_hi)
-        v = b_kmajor ? Bb[static_cast<long long>(gc) * ldb + gk] : Bb[static_cast<long long>(gk) * ldb + gc];
-      Bs[k][c] = v;
-    }
+    store_tiles(As, Bs, b_kmajor, tid, ra, rb);
     __syncthreads();
-#pragma unroll 8
-    for (int k = 0; k < TK; ++k) {
-      const float a0 = As[k][ty * 2], a1 = As[k][ty * 2 + 1];
-      const float b0 = Bs[k][tx * 2], b1 = Bs[k][tx * 2 + 1];
-      acc[0][0] = fmaf(a0, b0, acc[0][0]);
-      acc[0][1] = fmaf(a0, b1, acc[0][1]);
-      acc[1][0] = fmaf(a1, b0, acc[1][0]);
-      acc[1][1] = fmaf(a1, b1, acc[1][1]);
-    }
+    if (k0 + TK < k_hi) fetch_tiles(Ab, lda, Bb, ldb, b_kmajor, M, N, k_hi, m0, n0, k0 + TK, tid, ra, rb);
+    mult_slice(As, Bs, tx, ty, acc);
     __syncthreads();
   }
 #pragma unroll
@@ -149,8 +155,13 @@ __global__ void __launch_bounds__(256) simt_gemm_splitk_kernel(const float* __re
   for (int e = tid; e < rows * TN; e += 256) {
     const int rr = r * rows + e / TN, c = e % TN;
     const uint32_t off = static_cast<uint32_t>((rr * TN + c) * sizeof(float));
+    float pq[8];  // every slice's partial in flight at once, then summed in slice order
+#pragma unroll
+    for (int q = 0; q < 8; ++q) pq[q] = q < S ? ld_dsmem_f32(mapa_shared(base + off, static_cast<uint32_t>(q))) : 0.f;
     float v[1] = {0.f};
-    for (int q = 0; q < S; ++q) v[0] += ld_dsmem_f32(mapa_shared(base + off, static_cast<uint32_t>(q)));
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (q < S) v[0] += pq[q];
     if (n0 + c < N) epilogue_row<1>(epi, l, m0 + rr, n0 + c, v, M, N);
   }
   cluster_sync();  // no CTA leaves while another still reads its partial tile
@@ -169,7 +180,7 @@ cudaError_t launch_simt_gemm(const SimtGemm& g, cudaStream_t s) {
     sms = 148;
   }
   // split K over a cluster until the grid covers two CTAs per SM (each CTA
-  // holds 12.5 KB of shared memory and 32 registers per thread, so several
+  // holds 12.5 KB of shared memory and 64 registers per thread, so four
   // fit), keeping at least one TK-deep slice per CTA
   int S = 1;
   while (S < 8 && tiles * S < 2 * sms && g.K >= 2 * S * TK) S *= 2;
