@@ -57,8 +57,11 @@ def test_noalloc_matches_oracle_and_compute_update_twice(dmuon_lib, pdt, tol, ca
             assert torch.equal(B_new, B_ref[0])
 
 
-def test_noalloc_forced_resident_kernel(dmuon_lib):
-    _, Gs, Ms = make_inputs([(64, 256)], seed=105, m_std=1e-3)
+@pytest.mark.parametrize("shape", [(64, 256), (256, 1024), (1024, 256)], ids=["small", "medium", "medium-tall"])
+def test_noalloc_forced_resident_kernel(dmuon_lib, shape):
+    """A forced resident plan: the small-matrix kernel (64 x 256) and the
+    medium one (one CTA pair, Gram form; wide and tall storage)."""
+    _, Gs, Ms = make_inputs([shape], seed=105, m_std=1e-3)
     O_ref, _ = gpu_update(dmuon_lib, Gs, Ms, variant="batched")
     _, O_ora = oracle_update(Gs[0], Ms[0])
     for _ in range(2):
