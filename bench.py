@@ -554,8 +554,14 @@ def main():
         dom, dom_kernel, prof = pairk, "tc_gemm2_kernel (CTA pair)", "pair"
     elif gemm["launches"] > 0:
         dom, prof = gemm, None
-        dom_kernel = ("ns_small_kernel (resident)" if variants_used == {"batched"}
-                      else "tc_gemm_kernel / tc_gemm2_kernel / ns_small_kernel")
+        # a resident plan runs the small-matrix kernel (m <= 128, n <= 512) or
+        # the medium one (one CTA pair per matrix)
+        resident = {"ns_small_kernel" if int(e.split()[0]) <= 128 and int(e.split()[1]) <= 512 else "ns_mid_kernel"
+                    for e in plans if e.split()[4] == "batched"}
+        if variants_used == {"batched"}:
+            dom_kernel = " / ".join(sorted(resident)) + " (resident)"
+        else:
+            dom_kernel = " / ".join(["tc_gemm_kernel", "tc_gemm2_kernel"] + sorted(resident))
     else:
         dom, prof = simt, None
         dom_kernel = ("ns_f32_kernel (fp32 FFMA, every step in one cooperative launch)"
