@@ -242,28 +242,65 @@ __device__ __forceinline__ void box_rw(uint8_t* box, __nv_bfloat16* W, long long
   }
 }
 
+// The fused parameter write of a tile whose weight is stored transposed:
+// iterate element (row, col) is W[col][row].  Per 32-column chunk the warp
+// moves the 32 x 32 box of W (W rows col.., columns row0w..) through shared
+// memory: 16-byte coalesced loads, the update by one lane per W column,
+// 16-byte coalesced stores.  The boxes of the warp's chunks alternate
+// between two buffers, and each box is fetched with cp.async two chunks
+// ahead, so its load is in flight while the previous chunk is updated.
 template <int BN>
-__device__ __forceinline__ void apply_tile_transposed(const Epilogue& e, uint8_t* box, uint32_t tbase, int l, int row0w,
-                                                      int col0, int M, int N, int lane, int half) {
+__device__ __forceinline__ void apply_tile_transposed(const Epilogue& e, uint8_t* wstg, uint32_t tbase, int l,
+                                                      int row0w, int col0, int M, int N, int lane, int half) {
   float alpha = e.alpha, beta = e.beta;
   if (e.alpha_vec) alpha *= e.alpha_vec[l];
   if (e.beta_vec) beta *= e.beta_vec[l];
   __nv_bfloat16* W = static_cast<__nv_bfloat16*>(e.W[l]);
   const bool vec = ((reinterpret_cast<uintptr_t>(W) & 15) == 0) && ((e.ldw & 7) == 0);
   const int row = row0w + lane;
-  constexpr int NCH = BN / CH;
   constexpr int STRIDE = EPI_WARPS / 4;
+  constexpr int NT = BN / CH / STRIDE;  // chunks of this warp: half, half + STRIDE, ...
+  // W box of this warp's chunk t into buffer t & 1: asynchronous for whole
+  // 16-byte segments, plain loads for a ragged edge
+  auto fetch = [&](int t) {
+    const int col = col0 + (half + STRIDE * t) * CH;
+    if (col >= N || row0w >= M) return;
+    const int nrows = N - col < 32 ? N - col : 32;
+    const int ncols = M - row0w < 32 ? M - row0w : 32;
+    uint8_t* box = wstg + (t & 1) * WBOX;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int idx = q * 32 + lane;
+      const int br = idx >> 2, seg = idx & 3;
+      if (br >= nrows) continue;
+      const __nv_bfloat16* gp = W + static_cast<long long>(col + br) * e.ldw + row0w + seg * 8;
+      uint8_t* sp = box + br * 64 + seg * 16;
+      if (vec && seg * 8 + 8 <= ncols) {
+        cp_async16(smem_u32(sp), gp, 16);
+      } else {
+        __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(sp);
+        for (int k = 0; k < 8; ++k)
+          if (seg * 8 + k < ncols) h[k] = gp[k];
+      }
+    }
+  };
+  fetch(0);
+  cp_async_commit();
+  if (NT > 1) fetch(1);
+  cp_async_commit();
 #pragma unroll 1
-  for (int i = half; i < NCH; i += STRIDE) {
+  for (int t = 0; t < NT; ++t) {
+    const int i = half + STRIDE * t;
     const int col = col0 + i * CH;
     float v[32];
     tmem_ld_32cols(tbase + i * CH, v);  // warp-collective
-    if (col >= N || row0w >= M) continue;
+    cp_async_wait_group<1>();           // this chunk's box (one newer group may be pending)
+    __syncwarp();
+    uint8_t* box = wstg + (t & 1) * WBOX;
+    const bool live = col < N && row0w < M;
     const int nrows = N - col < 32 ? N - col : 32;     // W rows of the box
     const int ncols = M - row0w < 32 ? M - row0w : 32;  // W columns of the box
-    box_rw(box, W, e.ldw, col, row0w, nrows, ncols, vec, true, lane);
-    __syncwarp();
-    if (row < M) {
+    if (live && row < M) {
       __nv_bfloat16* bx = reinterpret_cast<__nv_bfloat16*>(box);
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
@@ -278,9 +315,12 @@ __device__ __forceinline__ void apply_tile_transposed(const Epilogue& e, uint8_t
       }
     }
     __syncwarp();
-    box_rw(box, W, e.ldw, col, row0w, nrows, ncols, vec, false, lane);
-    __syncwarp();  // the box is free for the next chunk
+    if (live) box_rw(box, W, e.ldw, col, row0w, nrows, ncols, vec, false, lane);
+    __syncwarp();  // the buffer is free: fetch the chunk after next into it
+    if (t + 2 < NT) fetch(t + 2);
+    cp_async_commit();
   }
+  cp_async_wait_group<0>();
 }
 
 long long tiles_per_matrix(int M, int N, int bm, int bn, bool sym) {
