@@ -314,6 +314,21 @@ PAIR_PROFILES = {"batch64-1024x1024-bf16": "tc_gemm_pair_batch64-1024x1024.md",
                  "llama8b-matrices-bf16": "tc_gemm_pair_llama8b-matrices.md"}
 
 
+def host_memory_short(bytes_per_rank: int, local_ranks: int):
+    """None when the host can pin bytes_per_rank for every rank of the node
+    (with a quarter of the available memory to spare), else the reason."""
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:  # no way to tell: try it
+        return None
+    need = bytes_per_rank * max(1, local_ranks)
+    if need * 1.25 <= avail:
+        return None
+    return (f"host memory: {need / 1e9:.1f} GB of pinned buffers for {local_ranks} rank(s), "
+            f"{avail / 1e9:.1f} GB available")
+
+
 def profile_traffic(kernel_file: Path, workload: str):
     """Per-launch DRAM traffic of the dominant kernel from the committed ncu
     summary of this workload, if it was taken on the current kernel source."""
@@ -496,35 +511,46 @@ def main():
     # dmuon_step_host_io: each step's gradients come from pinned host memory
     # and the updated parameters go back to pinned host memory; the library
     # pipelines both copies with the computation, chunk by chunk.
-    hG = [g.cpu().pin_memory() for g in Gs]
-    hW = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in Ws]
-    h2d = sum(x.numel() * x.element_size() for x in hG)
-    d2h = sum(x.numel() * x.element_size() for x in hW)
-    thG, thW = B.TensorList(hG), B.TensorList(hW)
+    # The pinned buffers are filled straight from the device (no pageable
+    # copy on the way); every rank of the node needs its own, so the leg is
+    # skipped, with the reason, when the host cannot hold them all.
+    h2d = sum(g.numel() * g.element_size() for g in Gs)
+    d2h = sum(x.numel() * x.element_size() for x in Ws)
+    e2e_skip = host_memory_short(h2d + d2h, int(os.environ.get("LOCAL_WORLD_SIZE", "1")))
+    if reduce_max([0.0 if e2e_skip is None else 1.0], ws, device=dev)[0] > 0 and e2e_skip is None:
+        e2e_skip = "host memory short on another rank of the node"  # every rank takes the same branch
+    e2e_ms = 0.0
+    if e2e_skip is None:
+        hG = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in Gs]
+        for hg, g in zip(hG, Gs):
+            hg.copy_(g)
+        hW = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in Ws]
+        thG, thW = B.TensorList(hG), B.TensorList(hW)
 
-    def step_io():
-        B.dmuon_step_host_io(tW, thG, tM, w.lr, w.wd, w.mu, w.ns_steps, params_host_out=thW, opts=opts,
-                             stream=stream)
+        def step_io():
+            B.dmuon_step_host_io(tW, thG, tM, w.lr, w.wd, w.mu, w.ns_steps, params_host_out=thW, opts=opts,
+                                 stream=stream)
 
-    for _ in range(2):  # plans of the host-I/O chunking
-        step_io()
+        for _ in range(2):  # plans of the host-I/O chunking
+            step_io()
     e2e_steps = max(3, min(args.steps, 20))
     barrier()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        step_io()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if e2e_skip is None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            step_io()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / e2e_steps
+        del hG, hW, thG, thW
 
     # ---------------- AdamW on the non-matrix parameters that train beside Muon
     # (a separate measurement, outside the step above): one 50304 x 1024
     # embedding table plus 96 vectors of 1024, in the workload's dtype, fp32
     # moments; 1.2 GB per launch (bf16) > L2.  Times dmuon_adamw_step alone.
     aw = adamw_measure(dev, stream, torch_dtype=wl.torch_dtype(w.param_dtype))
-    del hG, hW, thG, thW
 
     # ---------------- reduce over ranks (max), report on rank 0
     ms_max, e2e_max = reduce_max([ms, e2e_ms], ws, device=dev)
@@ -618,8 +644,10 @@ def main():
                       "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(aw["gbs"] / peaks["hbm_gbs"], 4),
                       "ms": round(aw["ms"], 4), "elements": aw["elements"], "bytes_per_element": aw["bpe"],
                       "set": "50304x1024 embedding + 96 x 1024 vectors"},
-            "e2e": {"value": round(job_value(e2e_max, 1, ws), 4), "unit": "ms", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
+            "e2e": ({"value": round(job_value(e2e_max, 1, ws), 4), "unit": "ms", "h2d_bytes_per_step": h2d,
+                     "d2h_bytes_per_step": d2h} if e2e_skip is None else
+                    {"value": None, "unit": "ms", "skipped": e2e_skip, "h2d_bytes_per_step": h2d,
+                     "d2h_bytes_per_step": d2h}),
             "gpu_launches": launches * args.steps,
             "gpu_launches_per_step": launches,
             "clocks": clk,

@@ -45,3 +45,15 @@ def test_profile_traffic_needs_matching_source(tmp_path, monkeypatch):
 
 def test_fp32_peak_from_unit_counts():
     assert bench.FP32_FFMA_TFLOPS == pytest.approx(148 * 128 * 2 * 1.965e9 / 1e12)
+
+
+def test_end_to_end_leg_skips_when_the_host_cannot_pin_every_rank():
+    """The end-to-end leg pins each rank's gradients and parameters; it is
+    skipped, with the reason, when the node's ranks together would not fit in
+    the host's available memory (with a quarter to spare)."""
+    import psutil
+    import bench
+    avail = psutil.virtual_memory().available
+    assert bench.host_memory_short(avail // 100, 2) is None
+    reason = bench.host_memory_short(avail, 8)
+    assert reason is not None and "8 rank(s)" in reason and "GB available" in reason
