@@ -203,11 +203,10 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_tall_kernel(const Momentu
 // Tall matrices, vector path (cols % 4 == 0, 16-byte aligned G and B):
 // 64 x 128 tiles.  Each warp reads 8 rows of the tile, a lane four
 // consecutive columns (one 16-byte load of B, one 8- or 16-byte load of G);
-// U goes to shared memory transposed, and each warp then writes rows of X
-// (stored columns) two elements per lane.  The shared tile is [128][64]
+// U goes to shared memory transposed, and each warp then writes 16 rows of
+// X (stored columns), eight elements per lane.  The shared tile is [128][64]
 // floats with the row index XOR-swizzled by an even key of the column, so
-// the transposed writes meet at most two lanes per bank and the 8-byte
-// reads of the write phase none.
+// the transposed writes meet at most two lanes per bank.
 constexpr int TVR = 64, TVC = 128;
 __device__ __forceinline__ int tv_idx(int c, int r) { return c * TVR + (r ^ (((c >> 2) & 15) << 1)); }
 
@@ -256,22 +255,38 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_tall_vec_kernel(const Mom
       for (int j = 0; j < 4; ++j) tile[tv_idx(4 * lane + j, rr)] = u[j];
     }
     __syncthreads();
-    // X rows c0..c0+127 (stored columns), columns r0..r0+63: lane takes two
-#pragma unroll 4
-    for (int k = 0; k < TVC / 8; ++k) {
-      const int cc = w + 8 * k;
-      const int xr = c0 + cc, xc = r0 + 2 * lane;
-      const float2 v = *reinterpret_cast<const float2*>(&tile[tv_idx(cc, 2 * lane)]);
-      if (xr < a.cols && xc < a.rows) {
-        const long long o = xoff + static_cast<long long>(xr) * a.ldx + xc;
-        if (xc + 1 < a.rows) {
-          if (a.x_f32)
-            *reinterpret_cast<float2*>(static_cast<float*>(a.X) + o) = v;
-          else
-            *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(a.X) + o) = __floats2bfloat162_rn(v.x, v.y);
+    // X rows c0..c0+127 (stored columns), columns r0..r0+63: a lane writes
+    // eight consecutive elements (16 bytes in bf16), eight lanes per X row,
+    // so one warp instruction covers four rows of 128 bytes.  The four rows
+    // of an instruction are 4 apart, so their swizzle keys differ and the
+    // shared-memory reads meet no more than two lanes per bank.
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int cc = 16 * w + 4 * (lane >> 3) + k, seg = lane & 7;
+      const int xr = c0 + cc, xc = r0 + 8 * seg;
+      if (xr >= a.cols || xc >= a.rows) continue;
+      float v[8];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const float2 t = *reinterpret_cast<const float2*>(&tile[tv_idx(cc, 8 * seg + 2 * p)]);
+        v[2 * p] = t.x;
+        v[2 * p + 1] = t.y;
+      }
+      const long long o = xoff + static_cast<long long>(xr) * a.ldx + xc;
+      if (xc + 8 <= a.rows) {
+        if (a.x_f32) {
+          float4* q = reinterpret_cast<float4*>(static_cast<float*>(a.X) + o);
+          q[0] = make_float4(v[0], v[1], v[2], v[3]);
+          q[1] = make_float4(v[4], v[5], v[6], v[7]);
         } else {
-          store_elem(a.X, o, v.x, a.x_f32);
+          uint4 u;
+          __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+          for (int t = 0; t < 4; ++t) h[t] = __floats2bfloat162_rn(v[2 * t], v[2 * t + 1]);
+          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.X) + o) = u;
         }
+      } else {
+        for (int t = 0; t < 8 && xc + t < a.rows; ++t) store_elem(a.X, o + t, v[t], a.x_f32);
       }
     }
     __syncthreads();
@@ -546,9 +561,9 @@ cudaError_t launch_momentum(const MomentumArgs& a, cudaStream_t s) {
   dim3 grid(a.nblk, a.cnt);
   if (a.transposed) {
     // the vector path reads four columns with one load: cols % 4 == 0 and
-    // 16-byte aligned G/B bases (a.aligned); X rows start 8-byte aligned
-    // (ldx % 8 == 0) for its two-element stores
-    if (a.cols % 4 == 0 && a.aligned && (a.ldx & 7) == 0)
+    // 16-byte aligned G/B bases (a.aligned); its eight-element X stores
+    // need 16-byte aligned rows (ldx % 8 == 0, X base 16-byte aligned)
+    if (a.cols % 4 == 0 && a.aligned && (a.ldx & 7) == 0 && (reinterpret_cast<uintptr_t>(a.X) & 15) == 0)
       momentum_tall_vec_kernel<<<grid, EW_THREADS, 0, s>>>(a);
     else
       momentum_tall_kernel<<<grid, EW_THREADS, 0, s>>>(a);
