@@ -296,7 +296,7 @@ def test_resident_medium_kernel(dmuon_lib, shapes):
         assert np.all(np.abs(to64(Wg[i]) - w_apply) <= np.abs(w_apply) * 2.0 ** -8 + terms * 1e-6), i
 
 
-@pytest.mark.parametrize("steps", [1, 2, 7])
+@pytest.mark.parametrize("steps", [0, 1, 2, 7])
 def test_resident_medium_steps(dmuon_lib, steps):
     shapes = [(256, 1024), (700, 180)]
     Ws, Gs, Ms = make_inputs(shapes, seed=98, m_std=1e-3)
