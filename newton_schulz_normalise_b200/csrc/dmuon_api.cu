@@ -577,7 +577,7 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
   constexpr int UP_A = 1, UP_B = 2, UP_OUT = 4;
   // The last product O = scale * Aop Bx (m x n, K = m, Bx the MN-major iterate),
   // once per orientation part with its epilogue.
-  auto final_product = [&](const void* Aop, const void* Bx, bool scale) -> int {
+  auto final_product = [&](const void* Aop, const void* Bx, bool scale, int aflags) -> int {
     return parts([&](int off, int nn, Epilogue fin) -> int {
       fin.alpha = 1.f;
       fin.alpha_vec = scale ? sv + off : nullptr;
@@ -586,7 +586,7 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
       fin.C = nullptr;
       return gemm(c, nn, f32, tile, false, static_cast<const uint8_t*>(Aop) + static_cast<size_t>(off) * sq * g.esz,
                   g.ldm, sq, static_cast<const uint8_t*>(Bx) + static_cast<size_t>(off) * sx * g.esz, g.ldx, sx, false,
-                  m, n, m, fin, s, UP_A);
+                  m, n, m, fin, s, aflags);
     });
   };
   if (variant == DMUON_VARIANT_GRAM) {
@@ -613,11 +613,14 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
       ep.sc = sq;
       ep.beta = h.b;
       ep.diag = h.a;
-      rc = gemm(c, cnt, f32, tile, true, A, g.ldm, sq, A, g.ldm, sq, false, m, m, m, ep, s, UP_A | UP_B | UP_OUT);
+      // Q_1 = P_0 is the last Q when there is one step: stored in full
+      rc = gemm(c, cnt, f32, tile, true, A, g.ldm, sq, A, g.ldm, sq, false, m, m, m, ep, s,
+                UP_A | UP_B | (h.steps == 1 ? 0 : UP_OUT));
       if (rc) return rc;
       if (k > 0) {  // Q_{k+1} = P_k Q_k
         rc = gemm(c, cnt, f32, tile, true, Pk, g.ldm, sq, Q[qi], g.ldm, sq, false, m, m, m,
-                  store_epi(Q[qi ^ 1], g.ldm, sq, f32, 1.f, nullptr), s, UP_A | UP_B | UP_OUT);
+                  store_epi(Q[qi ^ 1], g.ldm, sq, f32, 1.f, nullptr), s,
+                  UP_A | UP_B | (k == h.steps - 1 ? 0 : UP_OUT));
         if (rc) return rc;
         qi ^= 1;
       }
@@ -630,8 +633,9 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
         if (rc) return rc;
       }
     }
-    // O = s * Q_K U
-    return final_product(Q[qi], X0, true);
+    // O = s * Q_K U; Q_K is stored in full (its blocks below the diagonal
+    // mirrored), so the last and largest product reads it K-major
+    return final_product(Q[qi], X0, true, 0);
   }
   // ---------------- direct form
   // Per step: A = X X^T, P = c A^2 + b A + a I, X' = P X.  Folding a X into
@@ -659,7 +663,7 @@ int run_ns(DeviceCtx& c, const Chunk& ch, bool f32, int variant, int tile, const
     rc = gemm(c, cnt, f32, tile, true, A, g.ldm, sq, A, g.ldm, sq, false, m, m, m, ep, s, UP_A | UP_B | UP_OUT);
     if (rc) return rc;
     // X' = P X   (times s on the first step)
-    if (last) return final_product(P, cur, first);
+    if (last) return final_product(P, cur, first, UP_A);
     void* nxt = bufs[k & 1];
     rc = gemm(c, cnt, f32, tile, false, P, g.ldm, sq, cur, g.ldx, sx, false, m, n, m,
               store_epi(nxt, g.ldx, sx, f32, 1.f, first ? sv : nullptr), s, UP_A);
