@@ -1096,6 +1096,25 @@ int run_step(Request& r) {
     if (miss[x] != miss[y]) return static_cast<bool>(miss[x]);
     return group_cost(x) > group_cost(y);
   });
+  // the chunks in issue order, (group, first matrix of the chunk): group by
+  // group.  With host I/O and every plan cached, the chunks of all groups are
+  // merged instead, each group's spread evenly over the call (chunk i of a
+  // group of n chunks at (i + 1/2) / n).  A group's step is either copy-bound
+  // (a wide Gram group moves more bytes than it computes for) or
+  // compute-bound (a square direct one); run group by group, the copy
+  // engines idle through the compute-bound groups and the SMs through the
+  // copy-bound ones, while merged chunks keep both busy.
+  std::vector<std::pair<int, int>> seq;
+  for (int k : order)
+    for (int c0 = 0; c0 < static_cast<int>(groups[k].idx.size()); c0 += groups[k].chunk) seq.emplace_back(k, c0);
+  if (r.grads_host && !any_miss && groups.size() >= 2) {
+    auto pos = [&](const std::pair<int, int>& e) {
+      const Group& gr = groups[e.first];
+      const double n = static_cast<double>((gr.idx.size() + gr.chunk - 1) / gr.chunk);
+      return (e.second / gr.chunk + 0.5) / n;
+    };
+    std::stable_sort(seq.begin(), seq.end(), [&](const auto& x, const auto& y) { return pos(x) < pos(y); });
+  }
 
   // pointer tables, grouped: for group k, its matrices are contiguous.  With
   // host gradients the G entries point at the staging slot of the matrix's
@@ -1139,14 +1158,13 @@ int run_step(Request& r) {
       }
     }
     if (r.grads_host) {
-      int j = 0;
-      for (int k : order) {
+      for (size_t j = 0; j < seq.size(); ++j) {
+        const int k = seq[j].first, c0 = seq[j].second;
         const Group& gr = groups[k];
         const size_t stride = io_stride(gr.rows, gr.cols, g_f32);
         const int total = static_cast<int>(gr.idx.size());
-        for (int c0 = 0; c0 < total; c0 += gr.chunk, ++j)
-          for (int q = 0; q < std::min(gr.chunk, total - c0); ++q)
-            host[gstart[k] + c0 + q] = ws + stage_off + (j % io_slots) * align256(stage_slot) + q * stride;
+        for (int q = 0; q < std::min(gr.chunk, total - c0); ++q)
+          host[gstart[k] + c0 + q] = ws + stage_off + (j % io_slots) * align256(stage_slot) + q * stride;
       }
     }
   }
@@ -1170,11 +1188,12 @@ int run_step(Request& r) {
       if (side_used[i]) CUDA_TRY(cudaStreamWaitEvent(c.side[i], c.fork_ev, 0));
   }
 
-  for (int k : order) {
+  for (const auto& e : seq) {
+    const int k = e.first, c0 = e.second;
     Group& gr = groups[k];
     const Geo& g = geos[k];
     const int total = static_cast<int>(gr.idx.size());
-    for (int c0 = 0; c0 < total; c0 += gr.chunk) {
+    {
       const int ln = io_two ? (io_j & 1) : lane[k];
       const cudaStream_t gs = ln == 0 ? r.s : c.side[ln - 1];
       Chunk ch;
@@ -1247,7 +1266,7 @@ int run_step(Request& r) {
         ++io_j;
       }
     }
-    if (trace_on())
+    if (trace_on() && c0 + gr.chunk >= total)
       fprintf(stderr, "[dmuon] group %lldx%lld x%d (%d stored transposed): variant=%d tile=%d chunk=%d cost=%.3f ms stream=%d\n",
               gr.rows, gr.cols, total, gr.ntall, gr.plan.variant, gr.plan.tile, gr.chunk, gr.plan.cost_ms, lane[k]);
   }
