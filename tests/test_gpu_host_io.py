@@ -79,3 +79,31 @@ def test_host_io_pageable_and_unaligned_buffers(dmuon_lib):
         assert torch.equal(a, b)
     for i in range(len(shapes)):
         assert torch.equal(hW_mixed[i], mixed[0][i].cpu()), i
+
+
+def test_host_io_merged_chunks_match_group_order(dmuon_lib):
+    """Once every plan is cached, a host-I/O call issues the chunks of all its
+    shape groups interleaved (each group spread over the call) instead of
+    group by group.  The first call, which tunes and runs group by group, and
+    the second, merged, run the same plans on the same chunks: same bits."""
+    shapes = [(2048, 2048)] * 5 + [(1024, 4096)] * 4 + [(4096, 1024)] + [(512, 512)] * 3 + [(300, 130)] * 2
+    lr, wd, mu = 0.02, 0.1, 0.95
+    Ws, Gs, Ms = make_inputs(shapes, seed=80, m_std=1e-3)
+    W_ref, M_ref = gpu_step(dmuon_lib, Ws, Gs, Ms, lr, wd, mu)
+    hG = [g.cpu().pin_memory() for g in Gs]
+    runs = []
+    for _ in range(2):
+        W = [w.clone() for w in Ws]
+        M = [m.clone() for m in Ms]
+        hW = [torch.full(w.shape, float("nan"), dtype=w.dtype).pin_memory() for w in Ws]
+        dmuon_lib.dmuon_step_host_io(W, hG, M, lr, wd, mu, 5, params_host_out=hW)
+        torch.cuda.synchronize()
+        for i in range(len(shapes)):
+            assert torch.equal(hW[i], W[i].cpu()), i
+            assert torch.equal(M[i], M_ref[i]), i
+        runs.append(W)
+    for i, (r, c) in enumerate(shapes):
+        assert torch.equal(runs[0][i], runs[1][i]), i
+        d = np.linalg.norm(to64(runs[1][i]) - to64(W_ref[i]))
+        bound = lr * ora.rms_scale(r, c) * 6e-2 * np.sqrt(min(r, c)) + 2 ** -8 * np.linalg.norm(to64(W_ref[i]))
+        assert d <= bound, (i, d, bound)

@@ -272,8 +272,10 @@ def test_fp32_resident_nonfinite_stays_in_its_matrix(dmuon_lib):
 
 
 @pytest.mark.parametrize("shapes", [[(256, 1024)] * 3, [(200, 700)] * 2, [(1024, 256)], [(129, 300)], [(100, 900)],
-                                    [(200, 256)] * 2, [(250, 1000)]],
-                         ids=["256x1024x3", "200x700x2", "1024x256", "129x300", "100x900", "200x256x2", "250x1000"])
+                                    [(200, 256)] * 2, [(250, 1000)], [(1, 600)] * 2, [(3, 600)], [(700, 2)],
+                                    [(130, 513)], [(16, 1000), (1000, 16)]],
+                         ids=["256x1024x3", "200x700x2", "1024x256", "129x300", "100x900", "200x256x2", "250x1000",
+                              "1x600x2", "3x600", "700x2", "130x513", "16x1000-both"])
 def test_resident_medium_kernel(dmuon_lib, shapes):
     """The medium resident kernel (one CTA pair per matrix, the Gram-space
     chain on chip, X read twice, all steps in one launch) against the oracle
@@ -286,8 +288,13 @@ def test_resident_medium_kernel(dmuon_lib, shapes):
         _, Oo = oracle_update(Gs[i], Ms[i])
         assert rel_fro(to64(Ob[i]), Oo) <= BF16_TOL, (i, rel_fro(to64(Ob[i]), Oo))
         # near n = 1.25 m (200 x 256) both Gram forms sit 1.7e-2 from the
-        # oracle and 1.4e-2 from each other; elsewhere within 0.8e-2
-        assert rel_fro(to64(Ob[i]), to64(Og[i])) <= 2e-2, (i, rel_fro(to64(Ob[i]), to64(Og[i])))
+        # oracle and 1.4e-2 from each other; elsewhere within 0.8e-2.  An
+        # iterate of two or three rows has nearly equal singular values, and
+        # P = aI + bA + cA^2 is then dominated by its identity term: its bf16
+        # rounding keeps less of what tells its diagonal entries apart, and
+        # two bf16 forms drift further apart (up to 3e-2 in a CPU emulation).
+        x_tol = 2e-2 if min(shapes[i]) >= 16 else 3e-2
+        assert rel_fro(to64(Ob[i]), to64(Og[i])) <= x_tol, (i, rel_fro(to64(Ob[i]), to64(Og[i])))
         check_momentum(Bb[i], Gs[i], Ms[i], 0.95)
     Wg, _ = gpu_step(dmuon_lib, Ws, Gs, Ms, variant="batched")
     for i, (r, c) in enumerate(shapes):
