@@ -592,10 +592,16 @@ def main():
         dom, dom_kernel, prof = pairk, "tc_gemm2_kernel (CTA pair)", "pair"
     elif gemm["launches"] > 0:
         dom, prof = gemm, None
-        # a resident plan runs the small-matrix kernel (m <= 128, n <= 512) or
-        # the medium one (one CTA pair per matrix)
-        resident = {"ns_small_kernel" if int(e.split()[0]) <= 128 and int(e.split()[1]) <= 512 else "ns_mid_kernel"
-                    for e in plans if e.split()[4] == "batched"}
+        # a resident plan runs the small-matrix kernel (m <= 128, n <= 512),
+        # the medium one (one CTA pair per matrix), or for an fp32 iterate
+        # (iterates of at most 8 rows) the fp32 one
+        def resident_kernel(e):
+            f = e.split()
+            if f[2] == "f32":
+                return "ns_f32_kernel"
+            return "ns_small_kernel" if int(f[0]) <= 128 and int(f[1]) <= 512 else "ns_mid_kernel"
+
+        resident = {resident_kernel(e) for e in plans if e.split()[4] == "batched"}
         if variants_used == {"batched"}:
             dom_kernel = " / ".join(sorted(resident)) + " (resident)"
         else:

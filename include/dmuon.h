@@ -26,6 +26,12 @@
  *     candidate kernels are timed, the best is kept and reused for that shape.
  * The pages fix neither the coefficients nor eps; the defaults are
  * (a, b, c) = (3.4445, -4.7750, 2.0315), eps = 1e-7, K = 5.
+ * Precision: with bf16 parameters the iterate and the m x m matrices are
+ * rounded to bf16 between tensor-core products (fp32 accumulation, fp32
+ * epilogues), except that an iterate of at most 8 rows (min(rows, cols) <= 8)
+ * stays fp32 throughout on the CUDA cores: with so few, nearly equal
+ * singular values bf16 roundings would move O by several percent.  fp32
+ * parameters: fp32 throughout.
  *
  * Conventions for every entry point:
  *   - Device pointers are CUDA device memory of the current device; the
@@ -76,9 +82,10 @@ typedef enum dmuon_variant {
                                 to 8 small matrices per CTA, iterate, A and P in shared memory for
                                 all steps.  bf16, other m <= 256, n <= 1024 with 4n >= 5m: one CTA
                                 pair per matrix, the Gram-space chain (A, P, Q, m x m) in shared
-                                memory, X read twice.  fp32,
-                                m <= 1024: one cooperative launch over all SMs, a grid barrier
-                                between products.  Other shapes run as AUTO */
+                                memory, X read twice.  fp32 iterate (fp32
+                                parameters, or at most 8 rows), m <= 1024: one cooperative launch
+                                over all SMs, a grid barrier between products.  Other shapes run
+                                as AUTO */
 } dmuon_variant;
 
 /* Options of dmuon_step_ex.  Zero-initialise, then call dmuon_options_init. */
@@ -225,7 +232,9 @@ int dmuon_cache_load(const char* path);
 void dmuon_cache_clear(void);
 
 /* Number of cached shape keys, and the plan of key `i` as text
- * ("rows cols dtype variant bn chunk cost_ms") into buf (NUL-terminated). */
+ * ("rows cols dtype steps variant tile chunk cost_ms", dtype being the
+ * iterate's: "f32" for fp32 parameters and for iterates of at most 8 rows)
+ * into buf (NUL-terminated). */
 int dmuon_cache_size(void);
 int dmuon_cache_entry(int i, char* buf, size_t len);
 

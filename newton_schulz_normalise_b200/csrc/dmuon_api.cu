@@ -322,6 +322,17 @@ Geo make_geo(long long rows, long long cols, bool f32) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// The dtype of the Newton-Schulz iterate: the parameters' dtype, except that
+// bf16 weights whose iterate has at most kF32IterRows rows iterate in fp32.
+// A Gaussian iterate with two to eight rows has nearly equal normalised
+// singular values, which the five quintic steps still send to clearly
+// different values, so each bf16 rounding between the products turns the
+// singular vectors and moves the update by several percent (a CPU emulation
+// of the bf16 forms: up to 3.6% at 3 rows and 7% at 4 rows); products that
+// small leave the tensor cores idle anyway.
+constexpr long long kF32IterRows = 8;
+bool iter_f32(bool param_f32, long long m) { return param_f32 || m <= kF32IterRows; }
+
 // Scratch layout of one chunk of `cnt` matrices.
 struct Layout {
   size_t X0, Xp, Xq, A, Bm, P, Q0, Q1, T, partials, s, s2, sync, total;
@@ -684,6 +695,7 @@ struct Group {
   Plan plan;
   int chunk;
   int ntall;
+  bool xf = false;  // the iterate is fp32 (iter_f32)
 };
 
 struct Request {
@@ -997,16 +1009,18 @@ int run_step(Request& r) {
   size_t stage_slot = 0;  // host I/O: bytes of one staging slot for gradients
   for (size_t k = 0; k < groups.size(); ++k) {
     Group& gr = groups[k];
-    geos[k] = make_geo(gr.rows, gr.cols, f32);
+    gr.xf = iter_f32(f32, gr.rows);
+    geos[k] = make_geo(gr.rows, gr.cols, gr.xf);
     gr.chunk = chunk_size(geos[k], static_cast<int>(gr.idx.size()));
     if (r.grads_host) gr.chunk = std::min(gr.chunk, io_chunk(gr.rows, gr.cols, g_f32));
-    Key key{gr.rows, gr.cols, f32 ? 1 : 0, r.h.steps, gr.chunk};
+    Key key{gr.rows, gr.cols, gr.xf ? 1 : 0, r.h.steps, gr.chunk};
     {
       std::lock_guard<std::mutex> lk2(g_cache_mu);
       auto it = g_cache.find(key);
       // a forced variant the shape cannot take (see resident_supported)
       // runs as planned for AUTO
-      const bool forced_ok = r.o.variant != DMUON_VARIANT_BATCHED || resident_supported(f32, geos[k].m, geos[k].n);
+      const bool forced_ok =
+          r.o.variant != DMUON_VARIANT_BATCHED || resident_supported(gr.xf, geos[k].m, geos[k].n);
       const int want = forced_ok ? r.o.variant : DMUON_VARIANT_AUTO;
       if (it != g_cache.end() && (want == DMUON_VARIANT_AUTO || it->second.variant == want)) {
         gr.plan = it->second;
@@ -1038,7 +1052,7 @@ int run_step(Request& r) {
       const int tl = groups[k].plan.tile;
       const long long tiles = tc_gemm_tiles(g.m, g.n, groups[k].chunk, tl, false);
       const long long wave = tl >= 512 ? c.num_sms / 2 : c.num_sms;
-      if (groups[k].idx.size() <= static_cast<size_t>(groups[k].chunk) && tiles < 2 * wave)
+      if (!groups[k].xf && groups[k].idx.size() <= static_cast<size_t>(groups[k].chunk) && tiles < 2 * wave)
         small.push_back(static_cast<int>(k));
     }
     std::stable_sort(small.begin(), small.end(), [&](int x, int y) { return group_cost(x) > group_cost(y); });
@@ -1231,19 +1245,19 @@ int run_step(Request& r) {
         CUDA_TRY(cudaEventRecord(c.g_ready[slot], c.cin));
         CUDA_TRY(cudaStreamWaitEvent(gs, c.g_ready[slot], 0));
       }
-      rc = run_momentum(ch, f32, g_f32, r.h, gs);
+      rc = run_momentum(ch, gr.xf, g_f32, r.h, gs);
       if (rc) return rc;
       if (r.grads_host) CUDA_TRY(cudaEventRecord(c.g_free[slot], gs));
       if (miss[k] && c0 == 0) {
         Plan pl;
-        rc = autotune(c, ch, f32, r.h, r.o.variant, &pl, gs);
+        rc = autotune(c, ch, gr.xf, r.h, r.o.variant, &pl, gs);
         if (rc) return rc;
         gr.plan = pl;
-        Key key{gr.rows, gr.cols, f32 ? 1 : 0, r.h.steps, gr.chunk};
+        Key key{gr.rows, gr.cols, gr.xf ? 1 : 0, r.h.steps, gr.chunk};
         std::lock_guard<std::mutex> lk2(g_cache_mu);
         if (r.o.variant == DMUON_VARIANT_AUTO || !g_cache.count(key)) g_cache[key] = pl;
       }
-      rc = run_ns(c, ch, f32, gr.plan.variant, gr.plan.tile, r.h, final_epilogue(r, g, ch, f32, false),
+      rc = run_ns(c, ch, gr.xf, gr.plan.variant, gr.plan.tile, r.h, final_epilogue(r, g, ch, f32, false),
                   final_epilogue(r, g, ch, f32, true), ch.cnt, gs);
       if (rc) return rc;
       if (r.grads_host) {
@@ -1417,20 +1431,21 @@ int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows,
   int rc = validate(r);
   if (rc) return rc;
   const bool f32 = o.param_dtype == DMUON_F32;
+  const bool xf = iter_f32(f32, std::min(rows, cols));
   const bool tall = rows > cols;
-  const Geo g = make_geo(std::min(rows, cols), std::max(rows, cols), f32);  // the iterate, m x n
+  const Geo g = make_geo(std::min(rows, cols), std::max(rows, cols), xf);  // the iterate, m x n
   // plan: the resident kernel when it is asked for and the shape fits it;
   // else the plan the autotuner cached for this shape (count 1), else the
   // direct form (a forced variant the shape cannot take runs as AUTO)
   Plan plan;
-  if (o.variant == DMUON_VARIANT_BATCHED && resident_supported(f32, g.m, g.n)) {
+  if (o.variant == DMUON_VARIANT_BATCHED && resident_supported(xf, g.m, g.n)) {
     plan.variant = DMUON_VARIANT_BATCHED;
     plan.tile = 128;
   } else {
     const int want = o.variant == DMUON_VARIANT_BATCHED ? DMUON_VARIANT_AUTO : o.variant;
     if (want == DMUON_VARIANT_DIRECT || want == DMUON_VARIANT_GRAM) plan.variant = want;
     std::lock_guard<std::mutex> lk(g_cache_mu);
-    auto it = g_cache.find(Key{g.m, g.n, f32 ? 1 : 0, ns_steps, 1});
+    auto it = g_cache.find(Key{g.m, g.n, xf ? 1 : 0, ns_steps, 1});
     if (it != g_cache.end() && (want == DMUON_VARIANT_AUTO || it->second.variant == want)) plan = it->second;
   }
   void* base = nullptr;
@@ -1486,7 +1501,7 @@ int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows,
   ch.Ot = reinterpret_cast<float* const*>(dtab + 3);
   ch.nblk = nblk;
   ch.aligned = aligned16(grad) && aligned16(momentum);
-  rc = run_momentum(ch, f32, o.grad_dtype == DMUON_F32, r.h, s);
+  rc = run_momentum(ch, xf, o.grad_dtype == DMUON_F32, r.h, s);
   if (rc) return rc;
   Epilogue fin{};
   fin.mode = EPI_OUT;
@@ -1494,7 +1509,7 @@ int dmuon_compute_update_noalloc(const void* grad, void* momentum, int64_t rows,
   fin.transposed = tall ? 1 : 0;
   fin.ldw = tall ? g.m : g.n;
   fin.w_f32 = f32;
-  rc = run_ns(c, ch, f32, plan.variant, plan.tile, r.h, fin, fin, 1, s);
+  rc = run_ns(c, ch, xf, plan.variant, plan.tile, r.h, fin, fin, 1, s);
   if (rc) return rc;
   if (fault_wait()) {  // DMUON_FAULT=wait: a bounded wait that runs out, as a stalled pipeline would
     e = launch_wait_selftest(dev_err, 20000000ull, s);
@@ -1770,13 +1785,14 @@ int dmuon_workspace_size(const int64_t* shapes, int count, int param_dtype, size
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   cudaGetLastError();
   for (auto& kv : counts) {
-    Geo g = make_geo(kv.first.first, kv.first.second, f32);
+    const bool xf = iter_f32(f32, kv.first.first);
+    Geo g = make_geo(kv.first.first, kv.first.second, xf);
     const int total = kv.second.first + kv.second.second;
     int ch = chunk_size(g, total);
     Layout L = make_layout(g, ch, chunk_nblk(g, kv.second.first > 0, kv.second.second > 0));
     const size_t n_tune = align256(L.total + 2 * align256(static_cast<size_t>(ch) * g.x_elems() * g.esz) + 256);
     need = std::max(need, n_tune);
-    const bool maybe_small = !f32 && total <= ch && (tc_gemm_tiles(g.m, g.n, ch, 128, false) < 2LL * sms ||
+    const bool maybe_small = !xf && total <= ch && (tc_gemm_tiles(g.m, g.n, ch, 128, false) < 2LL * sms ||
                                                      tc_gemm_tiles(g.m, g.n, ch, 512, false) < sms);
     if (maybe_small) small_need = std::max(small_need, align256(L.total));
   }

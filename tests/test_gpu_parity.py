@@ -303,6 +303,29 @@ def test_resident_medium_kernel(dmuon_lib, shapes):
         assert np.all(np.abs(to64(Wg[i]) - w_apply) <= np.abs(w_apply) * 2.0 ** -8 + terms * 1e-6), i
 
 
+@pytest.mark.parametrize("shapes", [[(4, 1024)] * 3 + [(1024, 4)], [(3, 600)] * 5, [(8, 256)] * 40,
+                                    [(1, 64)] * 3 + [(5, 900), (2, 2)]],
+                         ids=["4x1024-both", "3x600x5", "8x256x40", "1x64-5x900-2x2"])
+def test_few_row_iterates_run_in_fp32(dmuon_lib, shapes):
+    """bf16 weights whose iterate has at most 8 rows iterate in fp32: with
+    so few, nearly equal singular values a bf16 iterate would move the update
+    by several percent.  Every variant meets the fp32 bar; the fused write
+    is the oracle's apply of the GPU's update within one bf16 rounding."""
+    Ws, Gs, Ms = make_inputs(shapes, seed=101, m_std=1e-3)
+    for variant in ("auto", "direct", "gram", "batched"):
+        Os, Bs = gpu_update(dmuon_lib, Gs, Ms, variant=variant)
+        for i in range(len(shapes)):
+            _, Oo = oracle_update(Gs[i], Ms[i])
+            assert rel_fro(to64(Os[i]), Oo) <= F32_TOL, (variant, i, rel_fro(to64(Os[i]), Oo))
+            check_momentum(Bs[i], Gs[i], Ms[i], 0.95)
+    Wg, _ = gpu_step(dmuon_lib, Ws, Gs, Ms)
+    for i, (r, c) in enumerate(shapes):
+        _, Oo = oracle_update(Gs[i], Ms[i])
+        w_apply = ora.apply_update(to64(Ws[i]), Oo, 0.02, 0.1)
+        terms = np.abs(0.998 * to64(Ws[i])) + np.abs(0.02 * ora.rms_scale(r, c) * Oo)
+        assert np.all(np.abs(to64(Wg[i]) - w_apply) <= np.abs(w_apply) * 2.0 ** -8 + terms * 1e-4), i
+
+
 @pytest.mark.parametrize("steps", [0, 1, 2, 7])
 def test_resident_medium_steps(dmuon_lib, steps):
     shapes = [(256, 1024), (700, 180)]
