@@ -594,7 +594,7 @@ def main():
         dom, prof = gemm, None
         # a resident plan runs the small-matrix kernel (m <= 128, n <= 512),
         # the medium one (one CTA pair per matrix), or for an fp32 iterate
-        # (iterates of at most 8 rows) the fp32 one
+        # (iterates of at most 5 rows) the fp32 one
         def resident_kernel(e):
             f = e.split()
             if f[2] == "f32":

@@ -28,7 +28,7 @@
  * (a, b, c) = (3.4445, -4.7750, 2.0315), eps = 1e-7, K = 5.
  * Precision: with bf16 parameters the iterate and the m x m matrices are
  * rounded to bf16 between tensor-core products (fp32 accumulation, fp32
- * epilogues), except that an iterate of at most 8 rows (min(rows, cols) <= 8)
+ * epilogues), except that an iterate of at most 5 rows (min(rows, cols) <= 5)
  * stays fp32 throughout on the CUDA cores: with so few, nearly equal
  * singular values bf16 roundings would move O by several percent.  fp32
  * parameters: fp32 throughout.
@@ -83,7 +83,7 @@ typedef enum dmuon_variant {
                                 all steps.  bf16, other m <= 256, n <= 1024 with 4n >= 5m: one CTA
                                 pair per matrix, the Gram-space chain (A, P, Q, m x m) in shared
                                 memory, X read twice.  fp32 iterate (fp32
-                                parameters, or at most 8 rows), m <= 1024: one cooperative launch
+                                parameters, or at most 5 rows), m <= 1024: one cooperative launch
                                 over all SMs, a grid barrier between products.  Other shapes run
                                 as AUTO */
 } dmuon_variant;
@@ -233,7 +233,7 @@ void dmuon_cache_clear(void);
 
 /* Number of cached shape keys, and the plan of key `i` as text
  * ("rows cols dtype steps variant tile chunk cost_ms", dtype being the
- * iterate's: "f32" for fp32 parameters and for iterates of at most 8 rows)
+ * iterate's: "f32" for fp32 parameters and for iterates of at most 5 rows)
  * into buf (NUL-terminated). */
 int dmuon_cache_size(void);
 int dmuon_cache_entry(int i, char* buf, size_t len);

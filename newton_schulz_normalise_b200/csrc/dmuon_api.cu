@@ -324,13 +324,14 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // The dtype of the Newton-Schulz iterate: the parameters' dtype, except that
 // bf16 weights whose iterate has at most kF32IterRows rows iterate in fp32.
-// A Gaussian iterate with two to eight rows has nearly equal normalised
+// A Gaussian iterate with three to five rows has nearly equal normalised
 // singular values, which the five quintic steps still send to clearly
 // different values, so each bf16 rounding between the products turns the
 // singular vectors and moves the update by several percent (a CPU emulation
-// of the bf16 forms: up to 3.6% at 3 rows and 7% at 4 rows); products that
-// small leave the tensor cores idle anyway.
-constexpr long long kF32IterRows = 8;
+// of the bf16 forms: up to 3.6% at 3 rows, 7.3% at 4 and 3.9% at 5; at most
+// 1.9% from 6 rows up); products that small leave the tensor cores idle
+// anyway.
+constexpr long long kF32IterRows = 5;
 bool iter_f32(bool param_f32, long long m) { return param_f32 || m <= kF32IterRows; }
 
 // Scratch layout of one chunk of `cnt` matrices.

@@ -303,11 +303,11 @@ def test_resident_medium_kernel(dmuon_lib, shapes):
         assert np.all(np.abs(to64(Wg[i]) - w_apply) <= np.abs(w_apply) * 2.0 ** -8 + terms * 1e-6), i
 
 
-@pytest.mark.parametrize("shapes", [[(4, 1024)] * 3 + [(1024, 4)], [(3, 600)] * 5, [(8, 256)] * 40,
+@pytest.mark.parametrize("shapes", [[(4, 1024)] * 3 + [(1024, 4)], [(3, 600)] * 5, [(5, 256)] * 40,
                                     [(1, 64)] * 3 + [(5, 900), (2, 2)]],
-                         ids=["4x1024-both", "3x600x5", "8x256x40", "1x64-5x900-2x2"])
+                         ids=["4x1024-both", "3x600x5", "5x256x40", "1x64-5x900-2x2"])
 def test_few_row_iterates_run_in_fp32(dmuon_lib, shapes):
-    """bf16 weights whose iterate has at most 8 rows iterate in fp32: with
+    """bf16 weights whose iterate has at most 5 rows iterate in fp32: with
     so few, nearly equal singular values a bf16 iterate would move the update
     by several percent.  Every variant meets the fp32 bar; the fused write
     is the oracle's apply of the GPU's update within one bf16 rounding."""
