@@ -136,9 +136,10 @@ int dmuon_step_ex(void* const* params, const void* const* grads, void* const* mo
  * (through four staging slots in the scratch) while a chunk is computed and
  * earlier chunks' parameters travel device->host.  Once every plan is
  * cached, consecutive chunks alternate between `stream` and an internal
- * compute stream, and the chunks of all shape groups run interleaved, each
- * group's spread evenly over the call, so that copy-bound chunks (wide
- * matrices) and compute-bound ones (square matrices) overlap.  Matrices of at most 256 KB whose host buffers are pinned
+ * compute stream; when one shape group is compute-bound (square matrices)
+ * and another copy-bound (wide ones), the chunks of the groups run
+ * interleaved, each group's spread evenly over the call, so that both kinds
+ * overlap.  Matrices of at most 256 KB whose host buffers are pinned
  * and 16-byte aligned are copied by a kernel that reads and writes the
  * mapped host memory, one launch per chunk; other matrices take one
  * copy-engine transfer each (DMUON_IO_COPY=dma|kernel forces one kind;

@@ -943,6 +943,7 @@ size_t io_stride(long long rows, long long cols, bool g_f32) {
 // DMUON_IO_COPY overrides.
 enum IoCopy { IO_AUTO = 0, IO_DMA = 1, IO_KERNEL = 2, IO_OUT_KERNEL = 3 };
 constexpr long long kIoKernelMaxBytes = 256 << 10;
+constexpr double kIoLinkGBs = 50.0;  // host link, GB/s per direction (PCIe 5 x16 measures about 56)
 IoCopy io_copy_mode() {
   static const IoCopy v = [] {
     const char* e = getenv("DMUON_IO_COPY");
@@ -1112,24 +1113,22 @@ int run_step(Request& r) {
     return group_cost(x) > group_cost(y);
   });
   // the chunks in issue order, (group, first matrix of the chunk): group by
-  // group.  With host I/O and every plan cached, the chunks of all groups are
-  // merged instead, each group's spread evenly over the call (chunk i of a
-  // group of n chunks at (i + 1/2) / n).  A group's step is either copy-bound
-  // (a wide Gram group moves more bytes than it computes for) or
-  // compute-bound (a square direct one); run group by group, the copy
-  // engines idle through the compute-bound groups and the SMs through the
-  // copy-bound ones, while merged chunks keep both busy.
+  // group.  With host I/O and every plan cached, when one group is
+  // copy-bound (a wide Gram group moves more bytes than it computes for) and
+  // another compute-bound (a square direct one), the chunks of the groups
+  // are merged instead, each group's spread evenly over the call (chunk i of
+  // a group of n chunks at (i + 1/2) / n): run group by group, the copy
+  // engines would idle through the compute-bound groups and the SMs through
+  // the copy-bound ones.  When every group is copy-bound the group order
+  // stays (merging measured slower there).
+  // Groups whose copies run through copy_tables_kernel are left out of the
+  // merge and follow the merged chunks, in group order: that kernel needs
+  // SMs, so between two big chunks it would wait for a GEMM to finish and
+  // hold up the copy stream behind it.  (The merge below runs once the copy
+  // kind of each group is known.)
   std::vector<std::pair<int, int>> seq;
   for (int k : order)
     for (int c0 = 0; c0 < static_cast<int>(groups[k].idx.size()); c0 += groups[k].chunk) seq.emplace_back(k, c0);
-  if (r.grads_host && !any_miss && groups.size() >= 2) {
-    auto pos = [&](const std::pair<int, int>& e) {
-      const Group& gr = groups[e.first];
-      const double n = static_cast<double>((gr.idx.size() + gr.chunk - 1) / gr.chunk);
-      return (e.second / gr.chunk + 0.5) / n;
-    };
-    std::stable_sort(seq.begin(), seq.end(), [&](const auto& x, const auto& y) { return pos(x) < pos(y); });
-  }
 
   // pointer tables, grouped: for group k, its matrices are contiguous.  With
   // host gradients the G entries point at the staging slot of the matrix's
@@ -1171,6 +1170,27 @@ int run_step(Request& r) {
         kin[k] = ok_in ? 1 : 0;
         kout[k] = ok_out ? 1 : 0;
       }
+    }
+    // The merge pays only when one group is compute-bound and another
+    // copy-bound: a chunk's measured compute time (its plan's cost) against
+    // its copies at a nominal host-link rate of kIoLinkGBs per direction.
+    bool compute_bound = false, copy_bound = false;
+    for (size_t k = 0; k < groups.size() && r.grads_host && !any_miss; ++k) {
+      if (kin[k] || kout[k]) continue;
+      const Group& gr = groups[k];
+      const double bytes = static_cast<double>(gr.chunk) * gr.rows * gr.cols *
+                           std::max(g_f32 ? 4 : 2, r.params_host ? (f32 ? 4 : 2) : 0);
+      (gr.plan.cost_ms > bytes / (kIoLinkGBs * 1e6) ? compute_bound : copy_bound) = true;
+    }
+    if (compute_bound && copy_bound) {
+      auto key = [&](const std::pair<int, int>& e) {
+        const Group& gr = groups[e.first];
+        if (kin[e.first] || kout[e.first]) return std::make_pair(1, 0.0);  // after the merged chunks, in order
+        const double n = static_cast<double>((gr.idx.size() + gr.chunk - 1) / gr.chunk);
+        return std::make_pair(0, (e.second / gr.chunk + 0.5) / n);
+      };
+      std::stable_sort(seq.begin(), seq.end(), [&](const auto& x, const auto& y) { return key(x) < key(y); });
+      if (trace_on()) fprintf(stderr, "[dmuon] host I/O: chunks merged across shape groups\n");
     }
     if (r.grads_host) {
       for (size_t j = 0; j < seq.size(); ++j) {

@@ -1,6 +1,12 @@
 """dmuon_step_host_io: gradients from pinned host memory, updated parameters
 copied back to host, copies pipelined with the computation.  Checked against
 dmuon_step on the same inputs and against the oracle."""
+import os
+import subprocess
+import sys
+import textwrap
+from pathlib import Path
+
 import numpy as np
 import pytest
 import torch
@@ -82,11 +88,13 @@ def test_host_io_pageable_and_unaligned_buffers(dmuon_lib):
 
 
 def test_host_io_merged_chunks_match_group_order(dmuon_lib):
-    """Once every plan is cached, a host-I/O call issues the chunks of all its
-    shape groups interleaved (each group spread over the call) instead of
-    group by group.  The first call, which tunes and runs group by group, and
-    the second, merged, run the same plans on the same chunks: same bits."""
-    shapes = [(2048, 2048)] * 5 + [(1024, 4096)] * 4 + [(4096, 1024)] + [(512, 512)] * 3 + [(300, 130)] * 2
+    """Once every plan is cached, a host-I/O call whose groups include a
+    compute-bound one (4096^2, direct form: 1.4 TFLOP per 33.5 MB) and a
+    copy-bound one (1024 x 4096, Gram form) issues their chunks interleaved
+    instead of group by group.  The first call, which tunes and runs group by
+    group, and the second, merged, run the same plans on the same chunks:
+    same bits."""
+    shapes = [(4096, 4096)] * 3 + [(1024, 4096)] * 4 + [(4096, 1024)] + [(512, 512)] * 3 + [(300, 130)] * 2
     lr, wd, mu = 0.02, 0.1, 0.95
     Ws, Gs, Ms = make_inputs(shapes, seed=80, m_std=1e-3)
     W_ref, M_ref = gpu_step(dmuon_lib, Ws, Gs, Ms, lr, wd, mu)
@@ -107,3 +115,35 @@ def test_host_io_merged_chunks_match_group_order(dmuon_lib):
         d = np.linalg.norm(to64(runs[1][i]) - to64(W_ref[i]))
         bound = lr * ora.rms_scale(r, c) * 6e-2 * np.sqrt(min(r, c)) + 2 ** -8 * np.linalg.norm(to64(W_ref[i]))
         assert d <= bound, (i, d, bound)
+
+
+@pytest.mark.parametrize("shapes,merged", [
+    ([(4096, 4096)] * 3 + [(1024, 4096)] * 4, True),      # compute-bound square group beside a copy-bound one
+    ([(1024, 4096)] * 4 + [(256, 1024)] * 64, False),     # every group copy-bound: group order stays
+], ids=["mixed", "all-copy-bound"])
+def test_host_io_merge_decision(shapes, merged):
+    """The chunks of a host-I/O call are merged across shape groups only when
+    one group is compute-bound and another copy-bound (checked through the
+    library's trace in a fresh process, after a first call that tunes)."""
+    script = f"""
+        import sys
+        sys.path[:0] = ["tests", "."]
+        import torch
+        from newton_schulz_normalise_b200 import binding as B
+        from parity_helpers import make_inputs
+        shapes = {shapes!r}
+        Ws, Gs, Ms = make_inputs(shapes, seed=81, m_std=1e-3)
+        hG = [g.cpu().pin_memory() for g in Gs]
+        hW = [torch.empty(w.shape, dtype=w.dtype).pin_memory() for w in Ws]
+        for i in range(2):
+            print("CALL", i, file=sys.stderr, flush=True)
+            B.dmuon_step_host_io(Ws, hG, Ms, 0.02, 0.1, 0.95, 5, params_host_out=hW)
+            torch.cuda.synchronize()
+    """
+    env = dict(os.environ, DMUON_TRACE="1")
+    r = subprocess.run([sys.executable, "-c", textwrap.dedent(script)], capture_output=True, text=True, timeout=300,
+                       cwd=Path(__file__).resolve().parents[1], env=env)
+    assert r.returncode == 0, r.stderr[-3000:]
+    second = r.stderr.split("CALL 1")[-1]
+    assert "CALL 0" in r.stderr and "chunks merged" not in r.stderr.split("CALL 1")[0]  # the first call tunes
+    assert ("chunks merged" in second) == merged, second[-2000:]
