@@ -1126,9 +1126,14 @@ int run_step(Request& r) {
   // SMs, so between two big chunks it would wait for a GEMM to finish and
   // hold up the copy stream behind it.  (The merge below runs once the copy
   // kind of each group is known.)
-  std::vector<std::pair<int, int>> seq;
-  for (int k : order)
-    for (int c0 = 0; c0 < static_cast<int>(groups[k].idx.size()); c0 += groups[k].chunk) seq.emplace_back(k, c0);
+  struct Piece {
+    int k, c0, cnt;  // group, its first matrix, matrices
+  };
+  std::vector<Piece> seq;
+  for (int k : order) {
+    const int n = static_cast<int>(groups[k].idx.size());
+    for (int c0 = 0; c0 < n; c0 += groups[k].chunk) seq.push_back({k, c0, std::min(groups[k].chunk, n - c0)});
+  }
 
   // pointer tables, grouped: for group k, its matrices are contiguous.  With
   // host gradients the G entries point at the staging slot of the matrix's
@@ -1183,23 +1188,40 @@ int run_step(Request& r) {
       (gr.plan.cost_ms > bytes / (kIoLinkGBs * 1e6) ? compute_bound : copy_bound) = true;
     }
     if (compute_bound && copy_bound) {
-      auto key = [&](const std::pair<int, int>& e) {
-        const Group& gr = groups[e.first];
-        if (kin[e.first] || kout[e.first]) return std::make_pair(1, 0.0);  // after the merged chunks, in order
+      auto key = [&](const Piece& e) {
+        const Group& gr = groups[e.k];
+        if (kin[e.k] || kout[e.k]) return std::make_pair(1, 0.0);  // after the merged chunks, in order
         const double n = static_cast<double>((gr.idx.size() + gr.chunk - 1) / gr.chunk);
-        return std::make_pair(0, (e.second / gr.chunk + 0.5) / n);
+        return std::make_pair(0, (e.c0 / gr.chunk + 0.5) / n);
       };
       std::stable_sort(seq.begin(), seq.end(), [&](const auto& x, const auto& y) { return key(x) < key(y); });
       if (trace_on()) fprintf(stderr, "[dmuon] host I/O: chunks merged across shape groups\n");
     }
+    // Host I/O with every plan cached: a quarter of the call's first chunk
+    // (at least one matrix) becomes a piece of its own, so the first
+    // computation starts after a short copy-in, and so does a quarter of the
+    // last chunk, so the last copy-out follows a short computation (the
+    // pipeline's fill and drain).  A piece runs its group's plan.
+    if (r.grads_host && !any_miss && !seq.empty()) {
+      auto split = [&](size_t i, bool head) {
+        const Piece e = seq[i];
+        if (e.cnt < 2) return;
+        const int a = std::max(1, e.cnt / 4);
+        const Piece x{e.k, e.c0, head ? a : e.cnt - a};
+        const Piece y{e.k, e.c0 + x.cnt, e.cnt - x.cnt};
+        seq[i] = x;
+        seq.insert(seq.begin() + static_cast<long>(i) + 1, y);
+      };
+      split(seq.size() - 1, false);
+      split(0, true);
+    }
     if (r.grads_host) {
       for (size_t j = 0; j < seq.size(); ++j) {
-        const int k = seq[j].first, c0 = seq[j].second;
-        const Group& gr = groups[k];
+        const Piece& e = seq[j];
+        const Group& gr = groups[e.k];
         const size_t stride = io_stride(gr.rows, gr.cols, g_f32);
-        const int total = static_cast<int>(gr.idx.size());
-        for (int q = 0; q < std::min(gr.chunk, total - c0); ++q)
-          host[gstart[k] + c0 + q] = ws + stage_off + (j % io_slots) * align256(stage_slot) + q * stride;
+        for (int q = 0; q < e.cnt; ++q)
+          host[gstart[e.k] + e.c0 + q] = ws + stage_off + (j % io_slots) * align256(stage_slot) + q * stride;
       }
     }
   }
@@ -1223,8 +1245,8 @@ int run_step(Request& r) {
       if (side_used[i]) CUDA_TRY(cudaStreamWaitEvent(c.side[i], c.fork_ev, 0));
   }
 
-  for (const auto& e : seq) {
-    const int k = e.first, c0 = e.second;
+  for (const Piece& e : seq) {
+    const int k = e.k, c0 = e.c0;
     Group& gr = groups[k];
     const Geo& g = geos[k];
     const int total = static_cast<int>(gr.idx.size());
@@ -1233,7 +1255,7 @@ int run_step(Request& r) {
       const cudaStream_t gs = ln == 0 ? r.s : c.side[ln - 1];
       Chunk ch;
       ch.g = &g;
-      ch.cnt = std::min(gr.chunk, total - c0);
+      ch.cnt = e.cnt;
       ch.nwide = std::min(std::max(total - gr.ntall - c0, 0), ch.cnt);
       ch.base = ws + region_off[ln];
       ch.nblk = chunk_nblk(g, gr.ntall < total, gr.ntall > 0);
@@ -1301,7 +1323,7 @@ int run_step(Request& r) {
         ++io_j;
       }
     }
-    if (trace_on() && c0 + gr.chunk >= total)
+    if (trace_on() && c0 + e.cnt >= total)
       fprintf(stderr, "[dmuon] group %lldx%lld x%d (%d stored transposed): variant=%d tile=%d chunk=%d cost=%.3f ms stream=%d\n",
               gr.rows, gr.cols, total, gr.ntall, gr.plan.variant, gr.plan.tile, gr.chunk, gr.plan.cost_ms, lane[k]);
   }
