@@ -136,7 +136,9 @@ int dmuon_step_ex(void* const* params, const void* const* grads, void* const* mo
  * (through four staging slots in the scratch) while a chunk is computed and
  * earlier chunks' parameters travel device->host.  Once every plan is
  * cached, consecutive chunks alternate between `stream` and an internal
- * compute stream; when one shape group is compute-bound (square matrices)
+ * compute stream, a quarter of the first and of the last chunk run as
+ * pieces of their own (a short pipeline fill and drain), and when one shape
+ * group is compute-bound (square matrices)
  * and another copy-bound (wide ones), the chunks of the groups run
  * interleaved, each group's spread evenly over the call, so that both kinds
  * overlap.  Matrices of at most 256 KB whose host buffers are pinned
