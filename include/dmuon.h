@@ -122,7 +122,8 @@ int dmuon_step(void* const* params, const void* const* grads, void* const* momen
 
 /* dmuon_step with explicit dtypes and options.  opts == NULL means defaults.
  * Supported: param/grad both BF16 (tensor-core path, bf16 operands, fp32
- * accumulate) or both F32 (fp32 SIMT path); momenta F32. */
+ * accumulate; an iterate of at most 5 rows in fp32 on the CUDA cores) or
+ * both F32 (fp32 SIMT path); momenta F32. */
 int dmuon_step_ex(void* const* params, const void* const* grads, void* const* momenta,
                   const int64_t* shapes, int count, float lr, float wd, float mu,
                   int ns_steps, const dmuon_options* opts, void* stream);
@@ -138,8 +139,8 @@ int dmuon_step_ex(void* const* params, const void* const* grads, void* const* mo
  * cached, consecutive chunks alternate between `stream` and an internal
  * compute stream, a quarter of the first and of the last chunk run as
  * pieces of their own (a short pipeline fill and drain), and when one shape
- * group is compute-bound (square matrices)
- * and another copy-bound (wide ones), the chunks of the groups run
+ * group is compute-bound (square matrices) and another copy-bound (wide
+ * ones), the chunks of the groups run
  * interleaved, each group's spread evenly over the call, so that both kinds
  * overlap.  Matrices of at most 256 KB whose host buffers are pinned
  * and 16-byte aligned are copied by a kernel that reads and writes the
