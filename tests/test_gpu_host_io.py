@@ -147,3 +147,27 @@ def test_host_io_merge_decision(shapes, merged):
     second = r.stderr.split("CALL 1")[-1]
     assert "CALL 0" in r.stderr and "chunks merged" not in r.stderr.split("CALL 1")[0]  # the first call tunes
     assert ("chunks merged" in second) == merged, second[-2000:]
+
+
+def test_host_io_few_row_groups_iterate_in_fp32(dmuon_lib):
+    """Host I/O with bf16 weights whose iterate has at most 5 rows (fp32
+    iterate) beside ordinary bf16 groups: the fp32 groups meet the fp32 bar,
+    the others the bf16 one, and the copied-out parameters are the device's."""
+    shapes = [(5, 700)] * 6 + [(1024, 3)] * 2 + [(6, 512)] * 4 + [(512, 1024)] * 3
+    Ws, Gs, Ms = make_inputs(shapes, seed=82, m_std=1e-3)
+    hG = [g.cpu().pin_memory() for g in Gs]
+    for call in range(2):  # the second call runs with cached plans (pieces, merge decision)
+        W = [w.clone() for w in Ws]
+        M = [m.clone() for m in Ms]
+        hW = [torch.empty(w.shape, dtype=w.dtype).pin_memory() for w in Ws]
+        dmuon_lib.dmuon_step_host_io(W, hG, M, 0.02, 0.1, 0.95, 5, params_host_out=hW)
+        torch.cuda.synchronize()
+        for i, (r, c) in enumerate(shapes):
+            assert torch.equal(hW[i], W[i].cpu()), (call, i)
+            _, Oo = ora.muon_update(to64(Gs[i]), to64(Ms[i]), 0.95, 5, 1e-7, True, "direct")
+            w_apply = ora.apply_update(to64(Ws[i]), Oo, 0.02, 0.1)
+            tol = 1e-4 if min(r, c) <= 5 else 3e-2
+            # the update's error budget plus one bf16 rounding of W'
+            budget = 0.02 * ora.rms_scale(r, c) * tol * np.linalg.norm(Oo) + 2 ** -8 * np.linalg.norm(w_apply)
+            d = np.linalg.norm(to64(W[i]) - w_apply)
+            assert d <= budget, (call, i, d, budget)
