@@ -316,6 +316,24 @@ int dmuon_adamw_step(void* const* params, const void* const* grads, float* const
  */
 int dmuon_selftest_wait(int limit_ms, void* stream);
 
+/*
+ * dmuon_debug_io_order -- the order in which a step issues its chunks, for a
+ * description of its shape groups: host logic only (no device work, no GPU
+ * needed), for tests of the scheduler.  Group g (listed in issue order, i.e.
+ * by descending measured cost) has counts[g] matrices in chunks of
+ * chunks[g], a measured chunk cost cost_ms[g] (ms), bytes[g] bytes per matrix
+ * over the host link (the larger direction) and sm_copy[g] != 0 when its
+ * host copies run through the copy kernel.  cached != 0 describes a
+ * dmuon_step_host_io call with every plan cached (chunks merged across
+ * groups when one is compute-bound and another copy-bound at a nominal
+ * 50 GB/s, the first and last chunks' quarters split off); cached = 0 any
+ * other call (group by group).  Writes up to `cap` pieces as (group, first
+ * matrix, matrices) int triples into `out` and returns the number of pieces;
+ * DMUON_ERR_INVALID on bad arguments.  The host arrays are the caller's.
+ */
+int dmuon_debug_io_order(const int* counts, const int* chunks, const double* cost_ms, const double* bytes,
+                         const int* sm_copy, int ngroups, int cached, int* out, int cap);
+
 /* Number of kernels the library launched since load (all kinds). */
 int64_t dmuon_launch_count(void);
 

@@ -33,7 +33,7 @@ EXPORTS = (
     "dmuon_cache_size", "dmuon_cache_entry", "dmuon_set_workspace", "dmuon_workspace_size",
     "dmuon_timing_enable", "dmuon_timing_reset", "dmuon_timing_get", "dmuon_launch_count",
     "dmuon_last_error", "dmuon_version", "dmuon_compute_update_noalloc", "dmuon_step_host_io",
-    "dmuon_selftest_wait", "dmuon_adamw_step",
+    "dmuon_selftest_wait", "dmuon_adamw_step", "dmuon_debug_io_order",
 )
 
 
@@ -58,6 +58,8 @@ def _load() -> ctypes.CDLL:
     P, I, F, I64, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int64, ctypes.c_size_t
     PP = ctypes.POINTER(ctypes.c_void_p)
     PI64 = ctypes.POINTER(ctypes.c_int64)
+    PI = ctypes.POINTER(ctypes.c_int)
+    PD = ctypes.POINTER(ctypes.c_double)
     sig = {
         "dmuon_options_init": (None, [ctypes.POINTER(Options)]),
         "dmuon_step": (I, [PP, PP, PP, PI64, I, F, F, F, I, P]),
@@ -82,6 +84,7 @@ def _load() -> ctypes.CDLL:
         "dmuon_step_host_io": (I, [PP, PP, PP, PP, PI64, I, F, F, F, I, ctypes.POINTER(Options), P]),
         "dmuon_selftest_wait": (I, [I, P]),
         "dmuon_adamw_step": (I, [PP, PP, PP, PP, PI64, I, F, F, F, F, F, I64, I, P]),
+        "dmuon_debug_io_order": (I, [PI, PI, PD, PD, PI, I, I, PI, I]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -344,6 +347,22 @@ def dmuon_selftest_wait(limit_ms: int = 50, stream=None) -> int:
     """Runs the bounded-wait self-test; returns the raw status (DMUON_ERR_DEVICE_TIMEOUT
     when the device-side timeout path works)."""
     return lib.dmuon_selftest_wait(limit_ms, _stream(stream))
+
+
+def dmuon_debug_io_order(groups, cached: bool):
+    """The chunk issue order of a step (host logic only): ``groups`` is a list
+    of (count, chunk, cost_ms, bytes_per_matrix, sm_copy) in issue order;
+    returns a list of (group, first matrix, matrices)."""
+    n = len(groups)
+    ints = lambda xs: (ctypes.c_int * max(n, 1))(*xs)  # noqa: E731
+    dbls = lambda xs: (ctypes.c_double * max(n, 1))(*xs)  # noqa: E731
+    args = (ints([g[0] for g in groups]), ints([g[1] for g in groups]), dbls([g[2] for g in groups]),
+            dbls([g[3] for g in groups]), ints([int(bool(g[4])) for g in groups]))
+    total = lib.dmuon_debug_io_order(*args, n, int(cached), None, 0)
+    _check(min(total, 0))
+    out = (ctypes.c_int * max(3 * total, 1))()
+    _check(min(lib.dmuon_debug_io_order(*args, n, int(cached), out, total), 0))
+    return [(out[3 * i], out[3 * i + 1], out[3 * i + 2]) for i in range(total)]
 
 
 def dmuon_launch_count() -> int:

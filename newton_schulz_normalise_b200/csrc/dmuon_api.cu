@@ -967,6 +967,72 @@ void* mapped_host(const void* p) {
   return a.devicePointer;
 }
 
+// The order in which a call issues its chunks.  Pure host logic: run_step
+// and dmuon_debug_io_order share it.
+struct IoGroup {
+  int count, chunk;  // matrices, matrices per chunk
+  double cost_ms;    // measured time of one chunk's computation (its plan's cost)
+  double bytes;      // bytes one matrix moves over the host link, the larger direction
+  bool sm_copy;      // its copies run through copy_tables_kernel
+};
+struct Piece {
+  int k, c0, cnt;  // group, its first matrix, matrices
+};
+// Group by group, in `order`, each group in chunks.  With host I/O and every
+// plan cached (io_cached):
+//  - when one group is copy-bound (a wide Gram group moves more bytes than it
+//    computes for) and another compute-bound (a square direct one), the
+//    chunks of the groups are merged, each group's spread evenly over the
+//    call (chunk i of a group of n chunks at (i + 1/2) / n): group by group,
+//    the copy engines would idle through the compute-bound groups and the
+//    SMs through the copy-bound ones.  A chunk's cost is compared with its
+//    copies at a nominal host-link rate of kIoLinkGBs per direction.  When
+//    every group is copy-bound the group order stays (merging measured
+//    slower there).  Groups copied through copy_tables_kernel stay out of the
+//    merge and follow the merged chunks, in group order: that kernel needs
+//    SMs, so between two big chunks it would wait for a GEMM to finish and
+//    hold up the copy stream behind it.
+//  - a quarter of the first chunk (at least one matrix) becomes a piece of
+//    its own, so the first computation starts after a short copy-in, and so
+//    does a quarter of the last chunk, so the last copy-out follows a short
+//    computation (the pipeline's fill and drain).  A piece runs its group's
+//    plan.
+std::vector<Piece> chunk_order(const std::vector<IoGroup>& gs, const std::vector<int>& order, bool io_cached,
+                               bool* merged) {
+  std::vector<Piece> seq;
+  for (int k : order)
+    for (int c0 = 0; c0 < gs[k].count; c0 += gs[k].chunk) seq.push_back({k, c0, std::min(gs[k].chunk, gs[k].count - c0)});
+  if (merged) *merged = false;
+  if (!io_cached || seq.empty()) return seq;
+  bool compute_bound = false, copy_bound = false;
+  for (const IoGroup& g : gs) {
+    if (g.sm_copy) continue;
+    (g.cost_ms > g.chunk * g.bytes / (kIoLinkGBs * 1e6) ? compute_bound : copy_bound) = true;
+  }
+  if (compute_bound && copy_bound) {
+    auto key = [&](const Piece& e) {
+      const IoGroup& g = gs[e.k];
+      if (g.sm_copy) return std::make_pair(1, 0.0);
+      const double n = static_cast<double>((g.count + g.chunk - 1) / g.chunk);
+      return std::make_pair(0, (e.c0 / g.chunk + 0.5) / n);
+    };
+    std::stable_sort(seq.begin(), seq.end(), [&](const Piece& x, const Piece& y) { return key(x) < key(y); });
+    if (merged) *merged = true;
+  }
+  auto split = [&](size_t i, bool head) {
+    const Piece e = seq[i];
+    if (e.cnt < 2) return;
+    const int a = std::max(1, e.cnt / 4);
+    const Piece x{e.k, e.c0, head ? a : e.cnt - a};
+    const Piece y{e.k, e.c0 + x.cnt, e.cnt - x.cnt};
+    seq[i] = x;
+    seq.insert(seq.begin() + static_cast<long>(i) + 1, y);
+  };
+  split(seq.size() - 1, false);
+  split(0, true);
+  return seq;
+}
+
 int run_step(Request& r) {
   int rc = validate(r);
   if (rc || r.count == 0) return rc;
@@ -1112,28 +1178,7 @@ int run_step(Request& r) {
     if (miss[x] != miss[y]) return static_cast<bool>(miss[x]);
     return group_cost(x) > group_cost(y);
   });
-  // the chunks in issue order, (group, first matrix of the chunk): group by
-  // group.  With host I/O and every plan cached, when one group is
-  // copy-bound (a wide Gram group moves more bytes than it computes for) and
-  // another compute-bound (a square direct one), the chunks of the groups
-  // are merged instead, each group's spread evenly over the call (chunk i of
-  // a group of n chunks at (i + 1/2) / n): run group by group, the copy
-  // engines would idle through the compute-bound groups and the SMs through
-  // the copy-bound ones.  When every group is copy-bound the group order
-  // stays (merging measured slower there).
-  // Groups whose copies run through copy_tables_kernel are left out of the
-  // merge and follow the merged chunks, in group order: that kernel needs
-  // SMs, so between two big chunks it would wait for a GEMM to finish and
-  // hold up the copy stream behind it.  (The merge below runs once the copy
-  // kind of each group is known.)
-  struct Piece {
-    int k, c0, cnt;  // group, its first matrix, matrices
-  };
-  std::vector<Piece> seq;
-  for (int k : order) {
-    const int n = static_cast<int>(groups[k].idx.size());
-    for (int c0 = 0; c0 < n; c0 += groups[k].chunk) seq.push_back({k, c0, std::min(groups[k].chunk, n - c0)});
-  }
+  std::vector<Piece> seq;  // the chunks in issue order (chunk_order), once the copy kinds are known
 
   // pointer tables, grouped: for group k, its matrices are contiguous.  With
   // host gradients the G entries point at the staging slot of the matrix's
@@ -1176,45 +1221,16 @@ int run_step(Request& r) {
         kout[k] = ok_out ? 1 : 0;
       }
     }
-    // The merge pays only when one group is compute-bound and another
-    // copy-bound: a chunk's measured compute time (its plan's cost) against
-    // its copies at a nominal host-link rate of kIoLinkGBs per direction.
-    bool compute_bound = false, copy_bound = false;
-    for (size_t k = 0; k < groups.size() && r.grads_host && !any_miss; ++k) {
-      if (kin[k] || kout[k]) continue;
+    std::vector<IoGroup> io(groups.size());
+    for (size_t k = 0; k < groups.size(); ++k) {
       const Group& gr = groups[k];
-      const double bytes = static_cast<double>(gr.chunk) * gr.rows * gr.cols *
-                           std::max(g_f32 ? 4 : 2, r.params_host ? (f32 ? 4 : 2) : 0);
-      (gr.plan.cost_ms > bytes / (kIoLinkGBs * 1e6) ? compute_bound : copy_bound) = true;
+      io[k] = {static_cast<int>(gr.idx.size()), gr.chunk, gr.plan.cost_ms,
+               static_cast<double>(gr.rows) * gr.cols * std::max(g_f32 ? 4 : 2, r.params_host ? (f32 ? 4 : 2) : 0),
+               kin[k] || kout[k]};
     }
-    if (compute_bound && copy_bound) {
-      auto key = [&](const Piece& e) {
-        const Group& gr = groups[e.k];
-        if (kin[e.k] || kout[e.k]) return std::make_pair(1, 0.0);  // after the merged chunks, in order
-        const double n = static_cast<double>((gr.idx.size() + gr.chunk - 1) / gr.chunk);
-        return std::make_pair(0, (e.c0 / gr.chunk + 0.5) / n);
-      };
-      std::stable_sort(seq.begin(), seq.end(), [&](const auto& x, const auto& y) { return key(x) < key(y); });
-      if (trace_on()) fprintf(stderr, "[dmuon] host I/O: chunks merged across shape groups\n");
-    }
-    // Host I/O with every plan cached: a quarter of the call's first chunk
-    // (at least one matrix) becomes a piece of its own, so the first
-    // computation starts after a short copy-in, and so does a quarter of the
-    // last chunk, so the last copy-out follows a short computation (the
-    // pipeline's fill and drain).  A piece runs its group's plan.
-    if (r.grads_host && !any_miss && !seq.empty()) {
-      auto split = [&](size_t i, bool head) {
-        const Piece e = seq[i];
-        if (e.cnt < 2) return;
-        const int a = std::max(1, e.cnt / 4);
-        const Piece x{e.k, e.c0, head ? a : e.cnt - a};
-        const Piece y{e.k, e.c0 + x.cnt, e.cnt - x.cnt};
-        seq[i] = x;
-        seq.insert(seq.begin() + static_cast<long>(i) + 1, y);
-      };
-      split(seq.size() - 1, false);
-      split(0, true);
-    }
+    bool merged = false;
+    seq = chunk_order(io, order, r.grads_host && !any_miss, &merged);
+    if (merged && trace_on()) fprintf(stderr, "[dmuon] host I/O: chunks merged across shape groups\n");
     if (r.grads_host) {
       for (size_t j = 0; j < seq.size(); ++j) {
         const Piece& e = seq[j];
@@ -1881,5 +1897,28 @@ int64_t dmuon_launch_count(void) { return g_launches.load(); }
 const char* dmuon_last_error(void) { return t_err.c_str(); }
 
 int dmuon_version(void) { return DMUON_VERSION; }
+
+int dmuon_debug_io_order(const int* counts, const int* chunks, const double* cost_ms, const double* bytes,
+                         const int* sm_copy, int ngroups, int cached, int* out, int cap) {
+  t_err.clear();
+  if (ngroups < 0 || cap < 0 || (cap > 0 && !out) ||
+      (ngroups > 0 && (!counts || !chunks || !cost_ms || !bytes || !sm_copy)))
+    return fail(DMUON_ERR_INVALID, "bad arguments");
+  std::vector<IoGroup> gs(ngroups);
+  std::vector<int> order(ngroups);
+  for (int g = 0; g < ngroups; ++g) {
+    if (counts[g] < 0 || chunks[g] < 1 || !std::isfinite(cost_ms[g]) || !std::isfinite(bytes[g]) || bytes[g] < 0)
+      return fail(DMUON_ERR_INVALID, "bad description of group %d", g);
+    gs[g] = {counts[g], chunks[g], cost_ms[g], bytes[g], sm_copy[g] != 0};
+    order[g] = g;
+  }
+  const std::vector<Piece> seq = chunk_order(gs, order, cached != 0, nullptr);
+  for (size_t i = 0; i < seq.size() && static_cast<long long>(i) < cap; ++i) {
+    out[3 * i] = seq[i].k;
+    out[3 * i + 1] = seq[i].c0;
+    out[3 * i + 2] = seq[i].cnt;
+  }
+  return static_cast<int>(seq.size());
+}
 
 }  // extern "C"
