@@ -317,6 +317,23 @@ int dmuon_adamw_step(void* const* params, const void* const* grads, float* const
 int dmuon_selftest_wait(int limit_ms, void* stream);
 
 /*
+ * dmuon_debug_groups -- the shape groups a step forms from `shapes` (count x 2
+ * int64, rows and cols per matrix): host logic only (no device work, no GPU
+ * needed), for tests of the grouping.  Matrices whose iterate is m x n
+ * (m = min, n = max of rows and cols) form one group, in order of first
+ * appearance.  For group g, out[6g .. 6g+5] = (m, n, matrices, matrices
+ * stored n x m, chunk, iterate in fp32 ? 1 : 0) for up to `cap` groups;
+ * `chunk` is the matrices per chain of launches (scratch within the
+ * workspace budget; with grads_host != 0, as for dmuon_step_host_io, also
+ * about DMUON_IO_CHUNK_MB of gradients).  If `members` is not NULL it
+ * receives the `count` matrix indices group by group, those stored m x n
+ * first.  Returns the number of groups; DMUON_ERR_INVALID for a bad shape or
+ * argument, DMUON_ERR_DTYPE for a bad param_dtype.
+ */
+int dmuon_debug_groups(const int64_t* shapes, int count, int param_dtype, int grads_host, int64_t* out, int cap,
+                       int* members);
+
+/*
  * dmuon_debug_io_order -- the order in which a step issues its chunks, for a
  * description of its shape groups: host logic only (no device work, no GPU
  * needed), for tests of the scheduler.  Group g (listed in issue order, i.e.

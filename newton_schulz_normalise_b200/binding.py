@@ -33,7 +33,7 @@ EXPORTS = (
     "dmuon_cache_size", "dmuon_cache_entry", "dmuon_set_workspace", "dmuon_workspace_size",
     "dmuon_timing_enable", "dmuon_timing_reset", "dmuon_timing_get", "dmuon_launch_count",
     "dmuon_last_error", "dmuon_version", "dmuon_compute_update_noalloc", "dmuon_step_host_io",
-    "dmuon_selftest_wait", "dmuon_adamw_step", "dmuon_debug_io_order",
+    "dmuon_selftest_wait", "dmuon_adamw_step", "dmuon_debug_io_order", "dmuon_debug_groups",
 )
 
 
@@ -85,6 +85,7 @@ def _load() -> ctypes.CDLL:
         "dmuon_selftest_wait": (I, [I, P]),
         "dmuon_adamw_step": (I, [PP, PP, PP, PP, PI64, I, F, F, F, F, F, I64, I, P]),
         "dmuon_debug_io_order": (I, [PI, PI, PD, PD, PI, I, I, PI, I]),
+        "dmuon_debug_groups": (I, [PI64, I, I, I, PI64, I, PI]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -347,6 +348,25 @@ def dmuon_selftest_wait(limit_ms: int = 50, stream=None) -> int:
     """Runs the bounded-wait self-test; returns the raw status (DMUON_ERR_DEVICE_TIMEOUT
     when the device-side timeout path works)."""
     return lib.dmuon_selftest_wait(limit_ms, _stream(stream))
+
+
+def dmuon_debug_groups(shapes, param_dtype=DMUON_BF16, grads_host=False):
+    """The shape groups a step forms (host logic only): a list of dicts with
+    m, n, count, ntall, chunk, iter_f32 and the member matrix indices."""
+    n = len(shapes)
+    arr = (ctypes.c_int64 * max(2 * n, 1))(*[v for s in shapes for v in s])
+    ng = lib.dmuon_debug_groups(arr, n, param_dtype, int(grads_host), None, 0, None)
+    _check(min(ng, 0))
+    out = (ctypes.c_int64 * max(6 * ng, 1))()
+    members = (ctypes.c_int * max(n, 1))()
+    _check(min(lib.dmuon_debug_groups(arr, n, param_dtype, int(grads_host), out, ng, members), 0))
+    res, pos = [], 0
+    for g in range(ng):
+        m, nn, cnt, ntall, chunk, xf = out[6 * g:6 * g + 6]
+        res.append({"m": m, "n": nn, "count": cnt, "ntall": ntall, "chunk": chunk, "iter_f32": bool(xf),
+                    "members": list(members[pos:pos + cnt])})
+        pos += cnt
+    return res
 
 
 def dmuon_debug_io_order(groups, cached: bool):

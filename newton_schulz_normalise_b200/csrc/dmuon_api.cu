@@ -19,6 +19,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <climits>
 #include <atomic>
 #include <cmath>
 #include <map>
@@ -967,6 +968,41 @@ void* mapped_host(const void* p) {
   return a.devicePointer;
 }
 
+// The shape groups of a call: the matrices whose iterate is m x n (m the
+// smaller, n the larger dimension, whichever way each is stored), in order of
+// first appearance, those stored m x n first (ntall stored n x m); per group
+// the iterate's dtype (iter_f32), its geometry and its chunk (matrices per
+// chain of launches: scratch within the workspace budget, and with host I/O
+// about DMUON_IO_CHUNK_MB of gradients).  Pure host logic: run_step and
+// dmuon_debug_groups share it.
+std::vector<Group> make_groups(const int64_t* shapes, int count, bool f32, bool io, bool g_f32,
+                               std::vector<Geo>* geos) {
+  std::vector<Group> groups;
+  std::map<std::pair<long long, long long>, int> gi;
+  for (int i = 0; i < count; ++i) {
+    const long long rr = shapes[2 * i], cc = shapes[2 * i + 1];
+    auto key = std::make_pair(std::min(rr, cc), std::max(rr, cc));
+    auto it = gi.find(key);
+    if (it == gi.end()) {
+      it = gi.emplace(key, static_cast<int>(groups.size())).first;
+      groups.push_back(Group{key.first, key.second, {}, Plan{}, 0, 0});
+    }
+    groups[it->second].idx.push_back(i);
+  }
+  geos->assign(groups.size(), Geo{});
+  for (size_t k = 0; k < groups.size(); ++k) {
+    Group& gr = groups[k];
+    auto tall = [&](int i) { return shapes[2 * i] > shapes[2 * i + 1]; };
+    std::stable_partition(gr.idx.begin(), gr.idx.end(), [&](int i) { return !tall(i); });
+    gr.ntall = static_cast<int>(std::count_if(gr.idx.begin(), gr.idx.end(), tall));
+    gr.xf = iter_f32(f32, gr.rows);
+    (*geos)[k] = make_geo(gr.rows, gr.cols, gr.xf);
+    gr.chunk = chunk_size((*geos)[k], static_cast<int>(gr.idx.size()));
+    if (io) gr.chunk = std::min(gr.chunk, io_chunk(gr.rows, gr.cols, g_f32));
+  }
+  return groups;
+}
+
 // The order in which a call issues its chunks.  Pure host logic: run_step
 // and dmuon_debug_io_order share it.
 struct IoGroup {
@@ -1048,39 +1084,15 @@ int run_step(Request& r) {
   const bool f32 = r.o.param_dtype == DMUON_F32;
   const bool g_f32 = r.o.grad_dtype == DMUON_F32;
 
-  // group by iterate shape (m, n), in order of first appearance; inside a
-  // group the matrices stored m x n come first
-  std::vector<Group> groups;
-  {
-    std::map<std::pair<long long, long long>, int> gi;
-    for (int i = 0; i < r.count; ++i) {
-      const long long rr = r.shapes[2 * i], cc = r.shapes[2 * i + 1];
-      auto key = std::make_pair(std::min(rr, cc), std::max(rr, cc));
-      auto it = gi.find(key);
-      if (it == gi.end()) {
-        it = gi.emplace(key, static_cast<int>(groups.size())).first;
-        groups.push_back(Group{key.first, key.second, {}, Plan{}, 0, 0});
-      }
-      groups[it->second].idx.push_back(i);
-    }
-    for (Group& gr : groups) {
-      auto tall = [&](int i) { return r.shapes[2 * i] > r.shapes[2 * i + 1]; };
-      std::stable_partition(gr.idx.begin(), gr.idx.end(), [&](int i) { return !tall(i); });
-      gr.ntall = static_cast<int>(std::count_if(gr.idx.begin(), gr.idx.end(), tall));
-    }
-  }
+  std::vector<Geo> geos;
+  std::vector<Group> groups = make_groups(r.shapes, r.count, f32, r.grads_host, g_f32, &geos);
   // plans: cache lookup; misses are tuned on this call's data below
-  std::vector<Geo> geos(groups.size());
   std::vector<bool> miss(groups.size(), false);
   std::vector<size_t> needs(groups.size(), 0);
   size_t ws_need = 0;
   size_t stage_slot = 0;  // host I/O: bytes of one staging slot for gradients
   for (size_t k = 0; k < groups.size(); ++k) {
     Group& gr = groups[k];
-    gr.xf = iter_f32(f32, gr.rows);
-    geos[k] = make_geo(gr.rows, gr.cols, gr.xf);
-    gr.chunk = chunk_size(geos[k], static_cast<int>(gr.idx.size()));
-    if (r.grads_host) gr.chunk = std::min(gr.chunk, io_chunk(gr.rows, gr.cols, g_f32));
     Key key{gr.rows, gr.cols, gr.xf ? 1 : 0, r.h.steps, gr.chunk};
     {
       std::lock_guard<std::mutex> lk2(g_cache_mu);
@@ -1897,6 +1909,36 @@ int64_t dmuon_launch_count(void) { return g_launches.load(); }
 const char* dmuon_last_error(void) { return t_err.c_str(); }
 
 int dmuon_version(void) { return DMUON_VERSION; }
+
+int dmuon_debug_groups(const int64_t* shapes, int count, int param_dtype, int grads_host, int64_t* out, int cap,
+                       int* members) {
+  t_err.clear();
+  if (count < 0 || (count > 0 && !shapes) || cap < 0 || (cap > 0 && !out))
+    return fail(DMUON_ERR_INVALID, "bad arguments");
+  if (param_dtype != DMUON_BF16 && param_dtype != DMUON_F32) return fail(DMUON_ERR_DTYPE, "bad dtype");
+  for (int i = 0; i < count; ++i)
+    if (shapes[2 * i] <= 0 || shapes[2 * i + 1] <= 0 || shapes[2 * i] > INT32_MAX || shapes[2 * i + 1] > INT32_MAX)
+      return fail(DMUON_ERR_INVALID, "bad shape of matrix %d", i);
+  const bool f32 = param_dtype == DMUON_F32;
+  std::vector<Geo> geos;
+  const std::vector<Group> groups = make_groups(shapes, count, f32, grads_host != 0, f32, &geos);
+  int pos = 0;
+  for (size_t k = 0; k < groups.size(); ++k) {
+    const Group& gr = groups[k];
+    if (static_cast<long long>(k) < cap) {
+      int64_t* o = out + 6 * k;
+      o[0] = gr.rows;
+      o[1] = gr.cols;
+      o[2] = static_cast<int64_t>(gr.idx.size());
+      o[3] = gr.ntall;
+      o[4] = gr.chunk;
+      o[5] = gr.xf ? 1 : 0;
+    }
+    if (members)
+      for (int i : gr.idx) members[pos++] = i;
+  }
+  return static_cast<int>(groups.size());
+}
 
 int dmuon_debug_io_order(const int* counts, const int* chunks, const double* cost_ms, const double* bytes,
                          const int* sm_copy, int ngroups, int cached, int* out, int cap) {
