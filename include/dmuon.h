@@ -319,7 +319,8 @@ int dmuon_selftest_wait(int limit_ms, void* stream);
 /*
  * dmuon_debug_groups -- the shape groups a step forms from `shapes` (count x 2
  * int64, rows and cols per matrix): host logic only (no device work, no GPU
- * needed), for tests of the grouping.  Matrices whose iterate is m x n
+ * needed), for tests of the grouping (DMuon release article, section 2:
+ * matrices are grouped by shape to feed the GPU).  Matrices whose iterate is m x n
  * (m = min, n = max of rows and cols) form one group, in order of first
  * appearance.  For group g, out[6g .. 6g+5] = (m, n, matrices, matrices
  * stored n x m, chunk, iterate in fp32 ? 1 : 0) for up to `cap` groups;
@@ -336,7 +337,8 @@ int dmuon_debug_groups(const int64_t* shapes, int count, int param_dtype, int gr
 /*
  * dmuon_debug_io_order -- the order in which a step issues its chunks, for a
  * description of its shape groups: host logic only (no device work, no GPU
- * needed), for tests of the scheduler.  Group g (listed in issue order, i.e.
+ * needed), for tests of the scheduler (DMuon release article, section 3:
+ * work is ordered by each shape group's measured cost).  Group g (listed in issue order, i.e.
  * by descending measured cost) has counts[g] matrices in chunks of
  * chunks[g], a measured chunk cost cost_ms[g] (ms), bytes[g] bytes per matrix
  * over the host link (the larger direction) and sm_copy[g] != 0 when its
